@@ -1,0 +1,155 @@
+"""CPU oracle for structured sparse causal attention with Fibonacci offsets.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg import this package; the library's product path
+never does, and it shares no code with the CUDA library.
+
+The arithmetic lives in ``oracle_attn.c`` (plain loops, see its header for the
+passages of "Depth-Staggered Fibonacci Spacing for Sparse Attention" it
+follows and the readings it takes).  This module only marshals numpy arrays.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+except the RoPE pairing convention (rotate-half versus interleaved pairs),
+which the page does not fix: parity unpinned for that choice alone.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from .build import build as _build
+
+FIB15 = (1, 2, 3, 5, 8, 13, 21, 34, 55, 89, 144, 233, 377, 610, 987)
+
+
+def _np_dtype(precision):
+    if precision == "f64":
+        return np.float64, ctypes.c_double
+    if precision == "f32":
+        return np.float32, ctypes.c_float
+    raise ValueError(precision)
+
+
+def _ptr(a, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _prep(x, dt):
+    return np.ascontiguousarray(np.asarray(x, dtype=dt))
+
+
+class Oracle:
+    """ctypes view of one build of oracle_attn.c (the default build, or a
+    deliberately mutated copy that the mutation tests compile)."""
+
+    def __init__(self, path):
+        lib = ctypes.CDLL(path)
+        for suffix, ctype in (("_f64", ctypes.c_double), ("_f32", ctypes.c_float)):
+            P = ctypes.POINTER(ctype)
+            head = [ctypes.c_int] * 7 + [ctypes.POINTER(ctypes.c_int32), ctypes.c_int,
+                                         ctypes.c_double, ctypes.c_double,
+                                         ctypes.POINTER(ctypes.c_float)]
+            fwd = getattr(lib, "oracle_fwd" + suffix)
+            fwd.restype = ctypes.c_int
+            fwd.argtypes = head + [P] * 6
+            bwd = getattr(lib, "oracle_bwd" + suffix)
+            bwd.restype = ctypes.c_int
+            bwd.argtypes = head + [P] * 8
+            geo = getattr(lib, "oracle_geometry" + suffix)
+            geo.restype = ctypes.c_int
+            geo.argtypes = [ctypes.c_float, ctypes.c_int32, ctypes.POINTER(ctypes.c_int64),
+                            ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
+            rope = getattr(lib, "oracle_rope" + suffix)
+            rope.restype = None
+            rope.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_double, P]
+        self.lib = lib
+        self.path = path
+
+    def fwd(self, q, k, v, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0,
+            scale=0.0, precision="f64", want_probs=False):
+        """Forward.  q, k, v: [L, B, H, T, D] (upcast); alpha: [L] fp32 values.
+
+        Returns (O, LSE) or (O, LSE, P), P [L, B, H, T, W+S+n_off] holding each
+        member's softmax weight in a fixed slot (window t, sink s, offset k),
+        0 where the member does not exist.
+        """
+        dt, ct = _np_dtype(precision)
+        q, k, v = (_prep(x, dt) for x in (q, k, v))
+        L, B, H, T, D = q.shape
+        assert k.shape == q.shape and v.shape == q.shape
+        al = _prep(alpha, np.float32).reshape(-1)
+        assert al.shape == (L,)
+        offs = np.ascontiguousarray(np.asarray(offsets, dtype=np.int32).reshape(-1))
+        o = np.empty_like(q)
+        lse = np.empty((L, B, H, T), dtype=dt)
+        n_slots = window + sinks + len(offs)
+        p = np.empty((L, B, H, T, n_slots), dtype=dt) if want_probs else None
+        fn = getattr(self.lib, "oracle_fwd_" + precision)
+        rc = fn(L, B, H, T, D, int(window), len(offs), _ptr(offs, ctypes.c_int32), int(sinks),
+                float(rope_base), float(scale), _ptr(al, ctypes.c_float),
+                _ptr(q, ct), _ptr(k, ct), _ptr(v, ct), _ptr(o, ct), _ptr(lse, ct),
+                _ptr(p, ct) if p is not None else None)
+        if rc != 0:
+            raise ValueError(f"oracle_fwd rejected its arguments (rc={rc})")
+        return (o, lse, p) if want_probs else (o, lse)
+
+    def bwd(self, q, k, v, dout, alpha, *, window, offsets=FIB15, sinks=0,
+            rope_base=10000.0, scale=0.0, precision="f64"):
+        """Backward for upstream dO: returns (dQ, dK, dV, dalpha[L])."""
+        dt, ct = _np_dtype(precision)
+        q, k, v, dout = (_prep(x, dt) for x in (q, k, v, dout))
+        L, B, H, T, D = q.shape
+        al = _prep(alpha, np.float32).reshape(-1)
+        assert al.shape == (L,)
+        offs = np.ascontiguousarray(np.asarray(offsets, dtype=np.int32).reshape(-1))
+        dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+        dal = np.empty((L,), dtype=dt)
+        fn = getattr(self.lib, "oracle_bwd_" + precision)
+        rc = fn(L, B, H, T, D, int(window), len(offs), _ptr(offs, ctypes.c_int32), int(sinks),
+                float(rope_base), float(scale), _ptr(al, ctypes.c_float),
+                _ptr(q, ct), _ptr(k, ct), _ptr(v, ct), _ptr(dout, ct),
+                _ptr(dq, ct), _ptr(dk, ct), _ptr(dv, ct), _ptr(dal, ct))
+        if rc != 0:
+            raise ValueError(f"oracle_bwd rejected its arguments (rc={rc})")
+        return dq, dk, dv, dal
+
+    def geometry(self, alpha, f):
+        """(ok, lo, w, c) of one offset under the oracle's reading."""
+        lo, w, c = ctypes.c_int64(), ctypes.c_double(), ctypes.c_int64()
+        ok = self.lib.oracle_geometry_f64(ctypes.c_float(alpha), int(f), ctypes.byref(lo),
+                                          ctypes.byref(w), ctypes.byref(c))
+        return bool(ok), lo.value, w.value, c.value
+
+    def rope(self, x, pos, rope_base=10000.0):
+        """RoPE of one row x[D] at integer position pos (fp64)."""
+        x = _prep(x, np.float64)
+        out = np.empty_like(x)
+        self.lib.oracle_rope_f64(_ptr(x, ctypes.c_double), int(pos), x.shape[0],
+                                 float(rope_base), _ptr(out, ctypes.c_double))
+        return out
+
+
+_default = None
+
+
+def default() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle(_build())
+    return _default
+
+
+def fwd(*a, **kw):
+    return default().fwd(*a, **kw)
+
+
+def bwd(*a, **kw):
+    return default().bwd(*a, **kw)
+
+
+def geometry(alpha, f):
+    return default().geometry(alpha, f)
+
+
+def rope(x, pos, rope_base=10000.0):
+    return default().rope(x, pos, rope_base)

@@ -1,0 +1,275 @@
+"""Pins of the CPU oracle against what the page and the mathematics fix.
+
+Every pin takes an ``Oracle`` instance, so the same checks run on the default
+build (tests/test_oracle_pins.py) and on deliberately mutated copies of the
+oracle's source (tests/test_oracle_mutants.py), which must each fail one pin.
+
+Page: "Depth-Staggered Fibonacci Spacing for Sparse Attention" (C. A. Capps),
+technical summary, Methodology ("Attended set", "Scaling", "Implementation")
+and "Experimental variables".
+"""
+import os
+
+import numpy as np
+
+from independent import dense_causal, integer_gather, multiset_bias, rope_complex
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def golden_offsets():
+    with open(os.path.join(GOLDEN, "fibonacci_offsets.txt")) as f:
+        rows = [ln for ln in f if ln.strip() and not ln.startswith("#")]
+    return tuple(int(x) for x in rows[0].split())
+
+
+def golden_alpha_schedules():
+    out = []
+    with open(os.path.join(GOLDEN, "alpha_schedules.txt")) as f:
+        for ln in f:
+            if ln.strip() and not ln.startswith("#"):
+                l, a, src = ln.split()
+                out.append((int(l), float(a), int(src)))
+    return out
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def _close(a, b, atol, rtol=0.0, what=""):
+    a, b = np.asarray(a), np.asarray(b)
+    err = np.abs(a - b)
+    lim = atol + rtol * np.abs(b)
+    assert np.all(err <= lim), f"{what}: max err {err.max():.3e} (limit {lim.max():.3e})"
+
+
+FIB = golden_offsets()
+
+
+# -- geometry ("Scaling": d_k = alpha f_k; interpolation and drop readings) ----
+
+def pin_geometry(orc):
+    for f in FIB:                       # integer alpha: no interpolation
+        assert orc.geometry(1.0, f) == (True, f, 0.0, f)
+        assert orc.geometry(2.0, f) == (True, 2 * f, 0.0, 2 * f)
+    assert orc.geometry(0.5, 1) == (True, 0, 0.5, 1)      # d = 0.5: rows i, i-1
+    assert orc.geometry(0.5, 2) == (True, 1, 0.0, 1)
+    assert orc.geometry(0.5, 3) == (True, 1, 0.5, 2)
+    assert orc.geometry(1.5, 987) == (True, 1480, 0.5, 1481)
+    assert orc.geometry(0.0, 5) == (True, 0, 0.0, 0)
+    for a in (np.float32(0.5 + 1 / 15), np.float32(1.1), np.float32(1.0333334)):
+        for f in FIB:                   # d is one fp32 product
+            d = np.float32(a) * np.float32(f)
+            lo = int(np.floor(d))
+            ok, glo, gw, gc = orc.geometry(float(a), f)
+            assert ok and glo == lo and gc == int(np.ceil(d))
+            assert gw == float(d - np.float32(lo))
+    for bad in (float("nan"), -1.0, 1e30):
+        assert not orc.geometry(bad, 3)[0]
+
+
+def pin_schedules():
+    """The golden schedule table against its stated closed forms."""
+    sched = golden_alpha_schedules()
+    assert [s[0] for s in sched] == list(range(16))
+    assert abs(sched[0][1] - 0.5) < 1e-15 and abs(sched[15][1] - 1.5) < 1e-15
+    for l, a, _ in sched:
+        assert abs(a - (0.5 + l / 15)) < 1e-15
+    src = [s[2] for s in sched]
+    assert sorted(src) == list(range(16))            # a permutation
+    assert all(src[src[l]] == l for l in range(16))  # 7*7 = 49 = 1 mod 16: self-inverse
+    assert FIB[:4] == (1, 2, 3, 5) and FIB[-1] == 987 and len(FIB) == 15
+    assert all(FIB[k + 1] == FIB[k] + FIB[k - 1] for k in range(1, 14))
+
+
+# -- RoPE ("RoPE before the gather") -------------------------------------------
+
+def pin_rope(orc):
+    x = _rand((16,), 1)
+    assert np.allclose(orc.rope(x, 0), x, atol=0, rtol=0)
+    for pos in (1, 7, 1000, 32767):
+        r = orc.rope(x, pos)
+        assert abs(np.linalg.norm(r) - np.linalg.norm(x)) < 1e-12
+        ref = rope_complex(np.stack([x] * (pos + 1)))[pos] if pos < 2000 else None
+        if ref is not None:
+            _close(r, ref, 1e-12, what="rope vs complex form")
+    # relative-position property: <R(q,i), R(k,j)> depends on i - j only
+    q, k = _rand((16,), 2), _rand((16,), 3)
+    base = orc.rope(q, 9) @ orc.rope(k, 4)
+    for s in (1, 50, 999):
+        assert abs(orc.rope(q, 9 + s) @ orc.rope(k, 4 + s) - base) < 1e-10
+    # frequencies: D=4, unit vector on dim 1 turns at theta_1 = base^(-1/2) = 0.01
+    e1 = np.array([0.0, 1.0, 0.0, 0.0])
+    for pos in (1, 3, 100):
+        r = orc.rope(e1, pos)
+        _close(r, [0.0, np.cos(0.01 * pos), 0.0, np.sin(0.01 * pos)], 1e-14, what="rope freq")
+
+
+# -- forward special cases -----------------------------------------------------
+
+def pin_dense_limit(orc):
+    """W >= T, no offsets, no sinks: plain dense causal attention."""
+    q, k, v = (_rand((1, 1, 2, 37, 8), s) for s in (10, 11, 12))
+    o, lse = orc.fwd(q, k, v, [1.0], window=37, offsets=())
+    o_ref, lse_ref = dense_causal(q, k, v)
+    _close(o, o_ref, 1e-12, what="dense O")
+    _close(lse, lse_ref, 1e-12, what="dense LSE")
+    o2, _ = orc.fwd(q, k, v, [1.0], window=50, offsets=(), scale=0.3)
+    _close(o2, dense_causal(q, k, v, scale=0.3)[0], 1e-12, what="dense O, scale")
+
+
+def pin_integer_gather(orc):
+    """alpha = 1 (and 2): the interpolated gather equals an exact integer gather."""
+    q, k, v = (_rand((1, 1, 2, 64, 16), s) for s in (20, 21, 22))
+    for alpha, sinks, window in ((1.0, 0, 6), (1.0, 4, 5), (2.0, 2, 3)):
+        o, lse = orc.fwd(q, k, v, [alpha], window=window, sinks=sinks, offsets=FIB)
+        o_ref, lse_ref = integer_gather(q, k, v, window=window, sinks=sinks,
+                                        dists=[int(alpha) * f for f in FIB])
+        _close(o, o_ref, 1e-12, what=f"integer gather O alpha={alpha}")
+        _close(lse, lse_ref, 1e-12, what=f"integer gather LSE alpha={alpha}")
+
+
+def pin_multiset(orc):
+    """Integer distances: the sparse set equals dense causal attention with a
+    log-multiplicity bias (duplicates from window/offset/sink overlaps kept)."""
+    T = 50
+    q, k, v = (_rand((1, 1, 1, T, 8), s) for s in (30, 31, 32))
+    for alpha, window, sinks in ((1.0, 4, 3), (1.0, 12, 0), (3.0, 2, 5)):
+        dists = [int(alpha) * f for f in FIB]
+        o, lse = orc.fwd(q, k, v, [alpha], window=window, sinks=sinks)
+        bias = multiset_bias(T, window=window, dists=dists, sinks=sinks)
+        o_ref, lse_ref = dense_causal(q, k, v, bias=bias)
+        _close(o, o_ref, 1e-12, what="multiset O")
+        _close(lse, lse_ref, 1e-12, what="multiset LSE")
+
+
+def pin_softmax(orc):
+    """Weights are >= 0 and sum to 1; members that do not exist weigh 0."""
+    q, k, v = (_rand((3, 1, 2, 40, 8), s) for s in (40, 41, 42))
+    alpha = np.float32([0.5, 1.0, 1.37])
+    W, S = 5, 2
+    _, _, p = orc.fwd(q, k, v, alpha, window=W, sinks=S, want_probs=True)
+    assert np.all(p >= 0)
+    _close(p.sum(-1), np.ones(p.shape[:-1]), 1e-12, what="sum p")
+    for i in range(40):
+        for t in range(W):                      # window slot t exists iff i-t >= 0
+            assert (p[..., i, t] > 0).all() == (i - t >= 0)
+        for s in range(S):
+            assert (p[..., i, W + s] > 0).all() == (s <= i)
+    # worked example, alpha = 1, query 2: offsets 1 and 2 exist, 3 is dropped
+    assert (p[1, ..., 2, W + S + 0] > 0).all() and (p[1, ..., 2, W + S + 1] > 0).all()
+    assert (p[1, ..., 2, W + S + 2:] == 0).all()
+    # alpha = 0.5: f=1 -> d=0.5 needs rows i and i-1, so it exists from i = 1
+    assert (p[0, ..., 0, W + S + 0] == 0).all() and (p[0, ..., 1, W + S + 0] > 0).all()
+
+
+def pin_constant_v(orc):
+    """Every V row equal to c: O = c, interpolated members included."""
+    q, k = (_rand((4, 1, 1, 60, 8), s) for s in (50, 51))
+    c = _rand((8,), 52)
+    v = np.broadcast_to(c, (4, 1, 1, 60, 8))
+    o, _ = orc.fwd(q, k, v, np.float32([0.5, 0.77, 1.21, 1.5]), window=3, sinks=1)
+    _close(o, np.broadcast_to(c, o.shape), 1e-12, what="constant V")
+
+
+def pin_interp_continuity(orc):
+    """As alpha*f approaches an integer n, the interpolated member approaches
+    the integer gather at distance n.  From below (lo = n-1, w -> 1) the weight
+    moves onto row i-n and the member exists from i = n, as in the integer
+    gather.  From above (lo = n, w -> 0) it needs row i-n-1, so by the drop
+    rule it exists only from i = n+1; at i = n the query sees the window alone.
+    Together these fix the direction of interpolation and the drop rule."""
+    q, k, v = (_rand((1, 1, 2, 30, 8), s) for s in (60, 61, 62))
+    f, n = 5, 7
+    o_int, _ = integer_gather(q, k, v, window=2, dists=[n])
+    o_win, _ = integer_gather(q, k, v, window=2, dists=[])
+    ref = {-1: o_int, 1: o_int.copy()}
+    ref[1][..., n, :] = o_win[..., n, :]
+    errs = {}
+    for eps in (1e-3, 1e-4):
+        for side in (-1, 1):
+            a = np.float32(n / f + side * eps)
+            o, _ = orc.fwd(q, k, v, [a], window=2, offsets=(f,))
+            errs[(eps, side)] = np.abs(o - ref[side]).max()
+    for side in (-1, 1):
+        assert errs[(1e-3, side)] < 0.05, errs
+        assert errs[(1e-4, side)] < errs[(1e-3, side)] / 4, errs   # O(eps) convergence
+
+
+def pin_nan_geometry(orc):
+    q, k, v = (_rand((2, 1, 1, 20, 8), s) for s in (70, 71, 72))
+    o, lse = orc.fwd(q, k, v, np.float32([np.nan, 1.0]), window=3)
+    assert np.isnan(o[0]).all() and np.isnan(lse[0]).all()
+    assert np.isfinite(o[1]).all() and np.isfinite(lse[1]).all()
+    o, _ = orc.fwd(q, k, v, np.float32([-1.0, 1.0]), window=3)
+    assert np.isnan(o[0]).all() and np.isfinite(o[1]).all()
+    dq, dk, dv, dal = orc.bwd(q, k, v, q, np.float32([np.nan, 1.0]), window=3)
+    assert np.isnan(dq[0]).all() and np.isnan(dk[0]).all() and np.isnan(dv[0]).all()
+    assert np.isnan(dal[0]) and np.isfinite(dal[1])
+
+
+def pin_fp32_build(orc):
+    """The fp32 build computes the same function to fp32 accuracy."""
+    q, k, v = (_rand((2, 1, 2, 64, 16), s) for s in (80, 81, 82))
+    al = np.float32([0.63, 1.47])
+    o64, l64 = orc.fwd(q, k, v, al, window=6, sinks=2)
+    o32, l32 = orc.fwd(q, k, v, al, window=6, sinks=2, precision="f32")
+    _close(o32, o64, 2e-6, what="fp32 O")
+    _close(l32, l64, 2e-6, what="fp32 LSE")
+    d64 = orc.bwd(q, k, v, o64, al, window=6, sinks=2)
+    d32 = orc.bwd(q, k, v, o64, al, window=6, sinks=2, precision="f32")
+    for a, b, name in zip(d32, d64, ("dq", "dk", "dv", "dalpha")):
+        _close(a, b, 5e-5, 1e-5, what=f"fp32 {name}")
+
+
+# -- backward (finite differences of sum(dO * O), fp64) ------------------------
+
+FD_ALPHA = np.float32([1.1234, 0.6789])   # every alpha*f (f*alpha <= 40) is >= 1e-2 from an integer
+FD_KW = dict(window=3, sinks=1)
+
+
+def _fd_problem():
+    shape = (2, 1, 2, 40, 8)
+    q, k, v, do = (_rand(shape, s) for s in (90, 91, 92, 93))
+    return q, k, v, do
+
+
+def pin_fd_inputs(orc):
+    q, k, v, do = _fd_problem()
+    dq, dk, dv, _ = orc.bwd(q, k, v, do, FD_ALPHA, **FD_KW)
+    h = 1e-6
+
+    def loss(qq, kk, vv):
+        return float((orc.fwd(qq, kk, vv, FD_ALPHA, **FD_KW)[0] * do).sum())
+
+    rng = np.random.default_rng(5)
+    for name, grad, which in (("dQ", dq, 0), ("dK", dk, 1), ("dV", dv, 2)):
+        idxs = [tuple(rng.integers(0, s) for s in q.shape) for _ in range(60)]
+        idxs += [(0, 0, 0, 0, 0), (1, 0, 1, 39, 7), (0, 0, 1, 1, 3)]
+        for idx in idxs:
+            args_p = [q.copy(), k.copy(), v.copy()]
+            args_m = [q.copy(), k.copy(), v.copy()]
+            args_p[which][idx] += h
+            args_m[which][idx] -= h
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - grad[idx]) <= 1e-6 + 1e-6 * abs(fd), (name, idx, fd, grad[idx])
+
+
+def pin_fd_alpha(orc):
+    q, k, v, do = _fd_problem()
+    _, _, _, dal = orc.bwd(q, k, v, do, FD_ALPHA, **FD_KW)
+    for l in range(2):
+        for h in (3e-4,):
+            ap, am = FD_ALPHA.copy(), FD_ALPHA.copy()
+            ap[l] = np.float32(FD_ALPHA[l] + h)
+            am[l] = np.float32(FD_ALPHA[l] - h)
+            lp = float((orc.fwd(q, k, v, ap, **FD_KW)[0] * do).sum())
+            lm = float((orc.fwd(q, k, v, am, **FD_KW)[0] * do).sum())
+            fd = (lp - lm) / (float(ap[l]) - float(am[l]))
+            assert abs(fd - dal[l]) <= 2e-3 * abs(fd) + 1e-6, (l, fd, dal[l])
+
+
+ALL_PINS = [pin_geometry, pin_rope, pin_dense_limit, pin_integer_gather, pin_multiset,
+            pin_softmax, pin_constant_v, pin_interp_continuity, pin_nan_geometry,
+            pin_fp32_build, pin_fd_inputs, pin_fd_alpha]
