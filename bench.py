@@ -1,0 +1,388 @@
+"""Benchmark of the structured sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...        # the CPU oracle as the reference arm
+
+One step is one pass of the whole path -- forward (offset geometry, RoPE,
+gather with interpolation, softmax, PV) and, for a training workload, the
+backward (dQ, dK, dV and the per-layer d-alpha) -- over one synthetic batch.
+The default workload is the learned-alpha training step: 16 layers, B=8, H=8,
+T=1024, d=64, W=12, bf16, forward plus backward.  With N GPUs every rank runs
+its own batch (independent (layer, batch, head) units: weak scaling, no
+collective on the data path); the step time is the max over ranks.
+
+Prints one JSON line (rank 0).  See the design doc for the byte counts behind the
+roofline figures.
+"""
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+METRIC = "sparse-attn fwd/bwd tokens·heads/s at T=1024/4096; HBM GB/s vs B200 peak"
+UNIT = "tokens·heads/s"
+FALLBACK_HBM_GBS = 6650.0
+
+# Algorithmic bytes per token-head for d=64 bf16 (2-byte elements, fp32 LSE / D):
+#   forward  : read Q, K, V; write O and LSE
+#   bwd query: read Q, K, V, O, dO, LSE; write dQ and D
+#   bwd key  : read Q, K, V, dO, LSE, D; write dK, dV
+# (the whole backward: Q, K, V, O, dO, dQ, dK, dV and LSE = 1028 B)
+def alg_bytes_per_token_head(kernel, D, elt):
+    row = D * elt
+    if kernel.startswith("fwd"):
+        return 4 * row + 4
+    if kernel.startswith("bwd_q"):
+        return 6 * row + 8
+    if kernel.startswith("bwd_kv"):
+        return 6 * row + 8
+    return 0
+
+
+# dram__bytes_read.sum + dram__bytes_write.sum per token-head from the ncu
+# captures summarised under profiles/, keyed by kernel and the hash of the
+# kernel sources they were taken on; a changed source reports null.
+MEASURED_TRAFFIC = {}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(HERE, "structured_sparse_attention_fibonacci_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:12]
+
+
+def measured_peaks():
+    path = os.path.join(HERE, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---- clocks during the timed region -----------------------------------------
+class ClockSampler:
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid=None):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 10:
+                continue
+            if self.uuid and parts[1] != self.uuid:
+                continue
+            try:
+                sm.append(float(parts[2]))
+                mx.append(float(parts[3]))
+                power.append(float(parts[4]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[6:10]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "power_w_max": max(power) if power else None,
+                "reasons": sorted(reasons)}
+
+
+# ---- multi-rank helpers (host logic; tested with gloo on CPU) --------------
+def max_over_ranks(value, device=None):
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(units_per_rank, world, steps, ms_max):
+    """Whole-job units per second: all ranks' units over the slowest rank's time."""
+    return units_per_rank * world * steps / (ms_max / 1e3)
+
+
+# ---- CPU baseline: the oracle as it stands, on a bounded sample -------------
+def oracle_sample(wl, budget_s):
+    """Time the fp32 oracle (forward, plus backward for training workloads) on
+    as many whole layers (all their (batch, head) units, OpenMP-parallel) as
+    fit the time budget; at least one layer."""
+    import oracle
+    from structured_sparse_attention_fibonacci_b200.inputs import make_inputs
+    kw = dict(window=wl.window, sinks=wl.sinks, offsets=wl.offsets, rope_base=wl.rope_base,
+              precision="f32")
+    alpha = wl.alpha().numpy()
+
+    def one_layer(l):
+        ts = make_inputs(wl, layers=range(l, l + 1))
+        arr = [t.float().numpy() for t in ts]
+        t0 = time.perf_counter()
+        oracle.fwd(arr[0], arr[1], arr[2], alpha[l:l + 1], **kw)
+        if wl.backward:
+            oracle.bwd(arr[0], arr[1], arr[2], arr[3], alpha[l:l + 1], **kw)
+        return time.perf_counter() - t0
+
+    t = one_layer(0)
+    n = 1
+    while n < wl.L and t * (n + 1) / n <= budget_s:
+        t += one_layer(n)
+        n += 1
+    cores = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+    units = n * wl.B * wl.H
+    sample = (f"{n} of {wl.L} layers = {units} (layer, batch, head) units "
+              f"({units * wl.T} token-heads), fp32 oracle "
+              f"{'forward+backward' if wl.backward else 'forward'}")
+    return {"value": units * wl.T / t, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": sample, "seconds": round(t, 3)}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle, timed on the host cores."""
+    from structured_sparse_attention_fibonacci_b200.inputs import WORKLOADS
+    if rank != 0:
+        return 0
+    wl = WORKLOADS[args.workload]
+    per_step_budget = max(1.0, args.reference_budget_s / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(wl, per_step_budget)
+    vals = [oracle_sample(wl, per_step_budget) for _ in range(args.steps)]
+    secs = sum(v["seconds"] for v in vals)
+    value = sum(v["value"] * v["seconds"] for v in vals) / secs
+    cb = dict(vals[-1])
+    cb["value"] = value
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / len(vals), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(wl, world), "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl, world):
+    return {"workload": wl.name, "L": wl.L, "B": wl.B, "H": wl.H, "T": wl.T, "D": wl.D,
+            "window": wl.window, "sinks": wl.sinks, "offsets": "fib15 (1..987)",
+            "alpha": wl.alpha_kind, "pass": "forward+backward" if wl.backward else "forward",
+            "global_batch": wl.B * world, "seq_len": wl.T, "parallelism": f"replicas{world}",
+            "l2": "inputs larger than L2 (no flush needed)"}
+
+
+# ---- our arm -------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import structured_sparse_attention_fibonacci_b200 as sa
+    from structured_sparse_attention_fibonacci_b200.inputs import WORKLOADS, make_inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.workload]
+    wl_rank = wl.shrink(seed=wl.seed + 100000 * rank) if world > 1 else wl
+    host = make_inputs(wl_rank, pin=True)
+    q, k, v = (t.to(dev) for t in host[:3])
+    do = host[3].to(dev) if wl.backward else None
+    alpha_h = wl.alpha().pin_memory()
+    alpha = alpha_h.to(dev)
+    kw = dict(window=wl.window, sinks=wl.sinks, offsets=wl.offsets, rope_base=wl.rope_base)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:4], dtype=torch.float32, device=dev)
+    if wl.backward:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+        dal = torch.empty(wl.L, dtype=torch.float32, device=dev)
+        ws = torch.empty(max(1, sa.workspace_size(tuple(q.shape), q.dtype, backward=True, **kw)),
+                         dtype=torch.uint8, device=dev)
+    launches = [0]
+
+    def step():
+        sa.fwd(q, k, v, alpha, out=o, lse=lse, **kw)
+        n = sa.last_launch_count()
+        if wl.backward:
+            sa.bwd(q, k, v, o, lse, do, alpha, dq=dq, dk=dk, dv=dv, dalpha=dal, workspace=ws, **kw)
+            n += sa.last_launch_count()
+        launches[0] += n
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.4)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches[0] = 0
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    gpu_launches = launches[0]
+    ms = e0.elapsed_time(e1)
+    ms_max = max_over_ranks(ms, dev)
+    value = aggregate_throughput(wl.token_heads, world, args.steps, ms_max)
+
+    # per-kernel times of the same steps (library trace: events on the launch stream)
+    sa.trace_enable(True)
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    trace = sa.trace_read()
+    sa.trace_enable(False)
+    kernels = {n: {"ms_per_launch": t / c, "launches": c} for n, (t, c) in trace.items()}
+    dominant = max(kernels, key=lambda n: kernels[n]["ms_per_launch"] * kernels[n]["launches"])
+    elt = 2 if wl.dtype == torch.bfloat16 else 4
+    peak, peak_kind = measured_peaks()
+    per_th = alg_bytes_per_token_head(dominant, wl.D, elt)
+    bytes_launch = per_th * wl.token_heads
+    achieved = bytes_launch / (kernels[dominant]["ms_per_launch"] / 1e3) / 1e9
+    key = f"{dominant}@{kernel_source_hash()}"
+    traffic = MEASURED_TRAFFIC.get(key)
+    roofline = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
+                "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                "alg_bytes_per_launch": bytes_launch,
+                "traffic": traffic * wl.token_heads if traffic is not None else None}
+    for n, kk in kernels.items():
+        b = alg_bytes_per_token_head(n, wl.D, elt) * wl.token_heads
+        kk["alg_GBps"] = b / (kk["ms_per_launch"] / 1e3) / 1e9 if b else None
+
+    # end to end through the public API: pinned host inputs in, results out
+    h_in = [t for t in host[:3]] + ([host[3]] if wl.backward else [])
+    d_in = [q, k, v] + ([do] if wl.backward else [])
+    outs = [o, lse] + ([dq, dk, dv, dal] if wl.backward else [])
+    h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in h_in) + alpha_h.numel() * 4
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+
+    def e2e_step():
+        for hs, ds in zip(h_in, d_in):
+            ds.copy_(hs, non_blocking=True)
+        alpha.copy_(alpha_h, non_blocking=True)
+        step()
+        for ho, do_ in zip(h_out, outs):
+            ho.copy_(do_, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), dev)
+    e2e = {"value": aggregate_throughput(wl.token_heads, world, args.steps, e2e_ms), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": e2e_ms / args.steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(wl, args.cpu_budget_s)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+                "config": workload_config(wl, world), "roofline": roofline,
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches, "clocks": clocks,
+                "kernels": kernels, "kernel_source": kernel_source_hash()}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="learned_train")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--reference-budget-s", type=float, default=120.0)
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

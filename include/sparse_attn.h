@@ -1,0 +1,154 @@
+/*
+ * sparse_attn.h -- C ABI of the structured sparse causal attention library
+ * (sm_100a / B200).
+ *
+ * The operation ("Depth-Staggered Fibonacci Spacing for Sparse Attention:
+ * Static Schedules Beat Learned Dilation and Extrapolate Where Dense
+ * Attention Fails", C. A. Capps; technical summary, section "Methodology"):
+ * for every layer l, batch b, head h and query position i, attention over
+ *   - the dense causal window  j = i, i-1, ..., i-W+1       ("Attended set"),
+ *   - S sink keys             j = 0 .. S-1 with j <= i     (optional),
+ *   - one member per offset f_k (the Fibonacci ladder 1, 2, 3, 5, ..., 987 by
+ *     default), at distance d_k = alpha_l * f_k             ("Scaling"),
+ *     linearly interpolated between rows when d_k is not an integer, with RoPE
+ *     applied to K (and Q) before the gather               ("Implementation").
+ * Exact arithmetic conventions (the library's reading of what the page leaves
+ * open):
+ *   d_k = fp32 product alpha_l * (float)f_k;  lo = floor(d_k);  w = d_k - lo;
+ *   offset k exists for query i iff i - ceil(d_k) >= 0;
+ *   key_k = (1-w) RoPE(K)[i-lo] + w RoPE(K)[i-lo-1], value_k likewise from V
+ *   (the second row is not read when w == 0);
+ *   q_hat_i = scale * RoPE(Q)[i]; score = q_hat_i . key; one softmax over all
+ *   members (duplicates are separate members); O_i = sum_m p_m value_m;
+ *   LSE_i = log sum_m exp(score_m);
+ *   RoPE: rotate-half pairs (j, j + D/2), angle pos * rope_base^(-2j/D), taken
+ *   in double precision and rounded to fp32;
+ *   an offset whose d_k lies outside [0, 2^24) (negative or NaN alpha, or one
+ *   so large that the product overflows the range) has no defined row: the
+ *   whole layer's outputs become NaN (no row is read for it).
+ *
+ * Tensors.  Q, K, V, O, dO, dQ, dK, dV are contiguous [L][B][H][T][D] arrays
+ * (D innermost) of the element type params.dtype, in DEVICE memory, 16-byte
+ * aligned.  LSE is a device fp32 [L][B][H][T] array; alpha and dalpha are
+ * device fp32 [L] arrays (these three need 4-byte alignment).  Accumulation is
+ * always fp32.
+ *
+ * Ownership.  The caller owns every buffer it passes (inputs, outputs and the
+ * workspace) and keeps them alive until the work queued on `stream` has
+ * finished.  On the first call for a given (device, T, D, rope_base) the
+ * library computes a RoPE cos/sin table on the device and keeps it, in memory
+ * it allocates once and releases at process exit; no other call allocates.
+ *
+ * Streams and errors.  Every call only enqueues kernels on `stream` (a
+ * cudaStream_t passed as void*, NULL = the legacy default stream) and returns
+ * without waiting.  Argument errors are detected on the host before anything
+ * is enqueued and return SA_ERR_INVALID_ARG / SA_ERR_UNSUPPORTED /
+ * SA_ERR_WORKSPACE; a failed launch returns SA_ERR_CUDA.  Nothing throws
+ * across this boundary and no call aborts the process.
+ */
+#ifndef SPARSE_ATTN_H
+#define SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, misaligned, f_k < 1, ... */
+  SA_ERR_UNSUPPORTED = 2,  /* valid but not built: D not in {16,32,64,128}, ... */
+  SA_ERR_WORKSPACE = 3,    /* workspace smaller than sparse_attn_workspace_size() */
+  SA_ERR_CUDA = 4,         /* a CUDA runtime call or a launch failed */
+  SA_ERR_INTERNAL = 5
+} sa_status;
+
+typedef enum { SA_DTYPE_F32 = 0, SA_DTYPE_BF16 = 1 } sa_dtype;
+
+/* Problem description.  All fields are read during the call only. */
+typedef struct {
+  int32_t L, B, H, T, D;   /* layers, batch, heads, sequence length, head dim   */
+  int32_t window;          /* W >= 1: keys i-W+1 .. i (the query itself included) */
+  int32_t n_offsets;       /* 0 .. SA_MAX_OFFSETS                                 */
+  const int32_t* offsets;  /* HOST array of n_offsets values f_k >= 1 (may be
+                              NULL when n_offsets == 0); copied during the call  */
+  int32_t n_sinks;         /* S >= 0: keys 0 .. S-1 always attended (when j <= i) */
+  float rope_base;         /* > 0, e.g. 10000                                     */
+  float scale;             /* score scale; <= 0 selects 1/sqrt(D)                 */
+  sa_dtype dtype;          /* element type of Q, K, V, O, dO, dQ, dK, dV          */
+} sa_params;
+
+#define SA_MAX_OFFSETS 32
+#define SA_MAX_SINKS 16
+
+/*
+ * Bytes of device workspace that sparse_attn_fwd (backward = 0) or
+ * sparse_attn_bwd (backward = 1) needs for these params; 0 when none.
+ * Returns 0 as well for invalid params (the call itself then reports why).
+ */
+size_t sparse_attn_workspace_size(const sa_params* p, int backward);
+
+/*
+ * Forward: O and (when lse != NULL) LSE for all L layers in one call.
+ *   q, k, v : device [L][B][H][T][D], dtype p->dtype           (read)
+ *   alpha   : device fp32 [L], the per-layer offset scale       (read)
+ *   o       : device [L][B][H][T][D], dtype p->dtype            (written)
+ *   lse     : device fp32 [L][B][H][T] or NULL                  (written)
+ *   workspace / workspace_bytes: device scratch of at least
+ *             sparse_attn_workspace_size(p, 0) bytes (may be NULL if 0).
+ * Source: "Depth-Staggered Fibonacci Spacing for Sparse Attention",
+ * Methodology -- "Attended set", "Scaling", "Implementation".
+ */
+sa_status sparse_attn_fwd(const sa_params* p, const void* q, const void* k, const void* v,
+                          const float* alpha, void* o, float* lse,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward of sparse_attn_fwd for the upstream gradient dout.
+ *   q, k, v, o, dout : device [L][B][H][T][D], dtype p->dtype   (read)
+ *   lse              : device fp32 [L][B][H][T] from the forward (read)
+ *   alpha            : device fp32 [L]                          (read)
+ *   dq, dk, dv       : device [L][B][H][T][D], dtype p->dtype   (overwritten)
+ *   dalpha           : device fp32 [L], overwritten with
+ *                      sum over (b, h, i, k) of dLoss/dw_k * f_k, the gradient
+ *                      to alpha through the interpolation weight w_k (floor
+ *                      held fixed: at an integer d_k this is the derivative
+ *                      from above; a second row i-lo-1 < 0 contributes 0).
+ *   workspace        : at least sparse_attn_workspace_size(p, 1) bytes.
+ * No atomics: every output element is written by exactly one thread and the
+ * per-layer dalpha is summed in a fixed order, so results are deterministic.
+ * Source: same passages; the page states that the interpolation lets
+ * gradients reach alpha ("Implementation") and trains alpha per layer
+ * ("Experimental variables", learned schedule).
+ */
+sa_status sparse_attn_bwd(const sa_params* p, const void* q, const void* k, const void* v,
+                          const void* o, const float* lse, const void* dout,
+                          const float* alpha, void* dq, void* dk, void* dv, float* dalpha,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* sparse_attn_status_string(sa_status s);
+
+/* Number of kernel launches the most recent successful fwd/bwd call on this
+ * host thread enqueued (a diagnostic for counting launches). */
+int32_t sparse_attn_last_launch_count(void);
+
+/*
+ * Kernel tracing (diagnostics).  While enabled (on != 0), every kernel the
+ * library enqueues is bracketed by two CUDA events recorded on the same
+ * stream.  sparse_attn_trace_read waits for all recorded events, writes up to
+ * `max` entries (static kernel name, total milliseconds, launch count), returns
+ * the number of distinct kernels, and clears the record.  Tracing is process
+ * wide and off by default; it costs two event records per launch.
+ */
+void sparse_attn_trace_enable(int on);
+int32_t sparse_attn_trace_read(int32_t max, const char** names, double* total_ms,
+                               int32_t* counts);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_ATTN_H */

@@ -1,0 +1,201 @@
+"""Structured sparse causal attention with depth-staggered Fibonacci offsets,
+for B200 (sm_100a).
+
+Thin ctypes binding over the C ABI in ``include/sparse_attn.h`` (library
+``libsparse_attn.so`` built in-tree by ``build.py``).  This module only
+marshals arguments: every step of the computation runs in the library's CUDA
+kernels.  There is no CPU fallback; if the library is missing or no GPU is
+present, the calls raise.
+
+    O, lse = fwd(q, k, v, alpha, window=12)                 # [L, B, H, T, D]
+    dq, dk, dv, dalpha = bwd(q, k, v, O, lse, dO, alpha, window=12)
+
+Method: "Depth-Staggered Fibonacci Spacing for Sparse Attention" (C. A.
+Capps), technical summary, Methodology -- "Attended set", "Scaling",
+"Implementation".
+"""
+import ctypes
+import os
+
+import torch
+
+FIB15 = (1, 2, 3, 5, 8, 13, 21, 34, 55, 89, 144, 233, 377, 610, 987)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsparse_attn.so")
+
+SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA, SA_ERR_INTERNAL = range(6)
+SA_DTYPE_F32, SA_DTYPE_BF16 = 0, 1
+MAX_OFFSETS = 32
+MAX_SINKS = 16
+
+EXPORTED = ("sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_workspace_size",
+            "sparse_attn_status_string", "sparse_attn_last_launch_count",
+            "sparse_attn_trace_enable", "sparse_attn_trace_read")
+
+
+class SaParams(ctypes.Structure):
+    _fields_ = [("L", ctypes.c_int32), ("B", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("T", ctypes.c_int32), ("D", ctypes.c_int32), ("window", ctypes.c_int32),
+                ("n_offsets", ctypes.c_int32), ("offsets", ctypes.POINTER(ctypes.c_int32)),
+                ("n_sinks", ctypes.c_int32), ("rope_base", ctypes.c_float),
+                ("scale", ctypes.c_float), ("dtype", ctypes.c_int32)]
+
+
+class SparseAttnError(RuntimeError):
+    def __init__(self, fn, status, msg):
+        super().__init__(f"{fn}: {msg} (status {status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m structured_sparse_attention_fibonacci_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER(SaParams)
+        vp, fp = ctypes.c_void_p, ctypes.c_void_p
+        L.sparse_attn_workspace_size.restype = ctypes.c_size_t
+        L.sparse_attn_workspace_size.argtypes = [P, ctypes.c_int]
+        L.sparse_attn_fwd.restype = ctypes.c_int
+        L.sparse_attn_fwd.argtypes = [P, vp, vp, vp, fp, vp, fp, vp, ctypes.c_size_t, vp]
+        L.sparse_attn_bwd.restype = ctypes.c_int
+        L.sparse_attn_bwd.argtypes = [P, vp, vp, vp, vp, fp, vp, fp, vp, vp, vp, fp, vp,
+                                      ctypes.c_size_t, vp]
+        L.sparse_attn_status_string.restype = ctypes.c_char_p
+        L.sparse_attn_status_string.argtypes = [ctypes.c_int]
+        L.sparse_attn_last_launch_count.restype = ctypes.c_int32
+        L.sparse_attn_last_launch_count.argtypes = []
+        L.sparse_attn_trace_enable.restype = None
+        L.sparse_attn_trace_enable.argtypes = [ctypes.c_int]
+        L.sparse_attn_trace_read.restype = ctypes.c_int32
+        L.sparse_attn_trace_read.argtypes = [ctypes.c_int32, ctypes.POINTER(ctypes.c_char_p),
+                                             ctypes.POINTER(ctypes.c_double),
+                                             ctypes.POINTER(ctypes.c_int32)]
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().sparse_attn_status_string(status).decode()
+
+
+def _check(fn, status):
+    if status != SA_OK:
+        raise SparseAttnError(fn, status, status_string(status))
+
+
+def make_params(shape, dtype, *, window, offsets=FIB15, sinks=0, rope_base=10000.0, scale=0.0):
+    """Build the C parameter block (the offsets array is kept alive on it)."""
+    L_, B, H, T, D = shape
+    offs = (ctypes.c_int32 * max(1, len(offsets)))(*[int(x) for x in offsets])
+    if dtype == torch.float32:
+        dt = SA_DTYPE_F32
+    elif dtype == torch.bfloat16:
+        dt = SA_DTYPE_BF16
+    else:
+        raise TypeError(f"unsupported dtype {dtype}")
+    p = SaParams(L_, B, H, T, D, int(window), len(offsets), offs, int(sinks),
+                 float(rope_base), float(scale), dt)
+    p._keep = offs
+    return p
+
+
+def workspace_size(shape, dtype, *, backward, **kw) -> int:
+    p = make_params(shape, dtype, **kw)
+    return int(lib().sparse_attn_workspace_size(ctypes.byref(p), int(bool(backward))))
+
+
+def last_launch_count() -> int:
+    """Kernels enqueued by the latest fwd/bwd call on this thread."""
+    return int(lib().sparse_attn_last_launch_count())
+
+
+def trace_enable(on: bool = True) -> None:
+    """Bracket every library kernel with CUDA events (see sparse_attn_trace_read)."""
+    lib().sparse_attn_trace_enable(int(bool(on)))
+
+
+def trace_read(max_kernels: int = 32):
+    """{kernel name: (total ms, launches)} since the last read; waits for the GPU."""
+    n = max_kernels
+    names = (ctypes.c_char_p * n)()
+    ms = (ctypes.c_double * n)()
+    ct = (ctypes.c_int32 * n)()
+    k = lib().sparse_attn_trace_read(n, names, ms, ct)
+    return {names[i].decode(): (ms[i], ct[i]) for i in range(min(k, n))}
+
+
+def _stream_handle(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _check_tensors(shape, dtype, device, **named):
+    for name, t in named.items():
+        if t is None:
+            continue
+        if t.device != device or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous tensor on {device}")
+        if name in ("alpha", "dalpha", "lse"):
+            if t.dtype != torch.float32:
+                raise TypeError(f"{name} must be float32")
+        elif tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+            raise ValueError(f"{name} must be {dtype} of shape {tuple(shape)}")
+
+
+def fwd(q, k, v, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0, scale=0.0,
+        out=None, lse=None, want_lse=True, stream=None):
+    """Sparse attention forward over all layers: returns (O, LSE or None).
+
+    q, k, v: CUDA tensors [L, B, H, T, D] (bf16 or fp32, contiguous).
+    alpha: CUDA fp32 [L].  Output buffers may be passed in via out= / lse=.
+    """
+    shape, dtype, dev = tuple(q.shape), q.dtype, q.device
+    if lse is None and want_lse:
+        lse = torch.empty(shape[:4], dtype=torch.float32, device=dev)
+    out = torch.empty_like(q) if out is None else out
+    _check_tensors(shape, dtype, dev, q=q, k=k, v=v, o=out, alpha=alpha, lse=lse)
+    p = make_params(shape, dtype, window=window, offsets=offsets, sinks=sinks,
+                    rope_base=rope_base, scale=scale)
+    L = lib()
+    ws_n = int(L.sparse_attn_workspace_size(ctypes.byref(p), 0))
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=dev) if ws_n else None
+    st = L.sparse_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(out),
+                           _ptr(lse), _ptr(ws), ws_n, _stream_handle(stream))
+    _check("sparse_attn_fwd", st)
+    return out, lse
+
+
+def bwd(q, k, v, o, lse, dout, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0,
+        scale=0.0, dq=None, dk=None, dv=None, dalpha=None, workspace=None, stream=None):
+    """Sparse attention backward: returns (dQ, dK, dV, dalpha[L])."""
+    shape, dtype, dev = tuple(q.shape), q.dtype, q.device
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    dalpha = torch.empty(shape[0], dtype=torch.float32, device=dev) if dalpha is None else dalpha
+    _check_tensors(shape, dtype, dev, q=q, k=k, v=v, o=o, dout=dout, dq=dq, dk=dk, dv=dv,
+                   alpha=alpha, dalpha=dalpha, lse=lse)
+    p = make_params(shape, dtype, window=window, offsets=offsets, sinks=sinks,
+                    rope_base=rope_base, scale=scale)
+    L = lib()
+    ws_n = int(L.sparse_attn_workspace_size(ctypes.byref(p), 1))
+    if workspace is None or workspace.numel() < ws_n:
+        workspace = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev)
+    st = L.sparse_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                           _ptr(dout), _ptr(alpha), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dalpha),
+                           _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check("sparse_attn_bwd", st)
+    return dq, dk, dv, dalpha

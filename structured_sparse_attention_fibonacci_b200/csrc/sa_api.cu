@@ -1,0 +1,225 @@
+// C ABI of the sparse-attention library: argument validation, workspace
+// sizing, the per-device RoPE table cache and kernel dispatch.  Declarations
+// and the contract (layouts, ownership, errors) are in include/sparse_attn.h.
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "sa_internal.h"
+#include "sparse_attn.h"
+
+namespace {
+
+thread_local int32_t g_last_launches = 0;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+sa_status build_problem(const sa_params* p, sa::Problem* pb) {
+  if (!p) return SA_ERR_INVALID_ARG;
+  if (p->L < 1 || p->B < 1 || p->H < 1 || p->T < 1) return SA_ERR_INVALID_ARG;
+  if (p->window < 1 || p->n_sinks < 0 || p->n_offsets < 0) return SA_ERR_INVALID_ARG;
+  if (p->n_offsets > SA_MAX_OFFSETS || p->n_sinks > SA_MAX_SINKS) return SA_ERR_UNSUPPORTED;
+  if (p->n_offsets > 0 && !p->offsets) return SA_ERR_INVALID_ARG;
+  if (!(p->rope_base > 0.f) || !isfinite(p->rope_base) || !isfinite(p->scale))
+    return SA_ERR_INVALID_ARG;
+  if (p->dtype != SA_DTYPE_F32 && p->dtype != SA_DTYPE_BF16) return SA_ERR_INVALID_ARG;
+  if (p->D != 16 && p->D != 32 && p->D != 64 && p->D != 128) return SA_ERR_UNSUPPORTED;
+  // index ranges: positions and per-unit offsets stay in int32, grids in 2^31
+  if (p->T > (1 << 24)) return SA_ERR_UNSUPPORTED;
+  const long long units = (long long)p->L * p->B * p->H;
+  if (units * (((long long)p->T + 15) / 16) >= (1LL << 31)) return SA_ERR_UNSUPPORTED;
+  pb->L = p->L; pb->B = p->B; pb->H = p->H; pb->T = p->T; pb->D = p->D;
+  pb->W = p->window; pb->n_off = p->n_offsets; pb->S = p->n_sinks;
+  pb->scale = p->scale > 0.f ? p->scale : (float)(1.0 / sqrt((double)p->D));
+  pb->dtype = p->dtype;
+  for (int k = 0; k < p->n_offsets; ++k) {
+    if (p->offsets[k] < 1) return SA_ERR_INVALID_ARG;
+    pb->f[k] = p->offsets[k];
+  }
+  return SA_OK;
+}
+
+// ---- RoPE cos/sin table, one per (device, D, base), grown on demand ---------
+struct RopeTable {
+  int dev, D;
+  float base;
+  int T_cap;
+  float2* ptr;
+};
+std::mutex g_rope_mu;
+std::vector<RopeTable> g_rope;  // superseded tables stay allocated until exit
+
+sa_status rope_table(int T, int D, float base, cudaStream_t st, const float2** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_rope_mu);
+  for (auto it = g_rope.rbegin(); it != g_rope.rend(); ++it) {
+    if (it->dev == dev && it->D == D && it->base == base && it->T_cap >= T) {
+      *out = it->ptr;
+      return SA_OK;
+    }
+  }
+  int cap = 4096;
+  while (cap < T) cap *= 2;
+  float2* ptr = nullptr;
+  if (cudaMalloc(&ptr, (size_t)cap * (D / 2) * sizeof(float2)) != cudaSuccess) return SA_ERR_CUDA;
+  if (sa::launch_rope_table(ptr, cap, D, (double)base, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaFree(ptr);
+    return SA_ERR_CUDA;
+  }
+  g_rope.push_back({dev, D, base, cap, ptr});
+  *out = ptr;
+  return SA_OK;
+}
+
+// ---- kernel tracing ---------------------------------------------------------
+struct TraceRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+std::mutex g_trace_mu;
+bool g_trace_on = false;
+std::vector<TraceRec> g_trace;       // completed begin/end pairs
+std::vector<cudaEvent_t> g_ev_pool;  // reusable events
+TraceRec g_open = {nullptr, nullptr, nullptr};
+
+cudaEvent_t take_event() {
+  if (!g_ev_pool.empty()) {
+    cudaEvent_t e = g_ev_pool.back();
+    g_ev_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+}  // namespace
+
+namespace sa {
+void trace_mark(const char* kernel, cudaStream_t st, bool begin) {
+  std::lock_guard<std::mutex> lock(g_trace_mu);
+  if (!g_trace_on) return;
+  cudaEvent_t e = take_event();
+  if (!e) return;
+  cudaEventRecord(e, st);
+  if (begin) {
+    g_open = {kernel, e, nullptr};
+  } else if (g_open.name == kernel) {
+    g_open.b = e;
+    g_trace.push_back(g_open);
+    g_open = {nullptr, nullptr, nullptr};
+  } else {
+    g_ev_pool.push_back(e);
+  }
+}
+}  // namespace sa
+
+extern "C" {
+
+const char* sparse_attn_status_string(sa_status s) {
+  switch (s) {
+    case SA_OK: return "ok";
+    case SA_ERR_INVALID_ARG: return "invalid argument";
+    case SA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SA_ERR_WORKSPACE: return "workspace too small";
+    case SA_ERR_CUDA: return "CUDA error";
+    case SA_ERR_INTERNAL: return "internal error";
+  }
+  return "unknown status";
+}
+
+int32_t sparse_attn_last_launch_count(void) { return g_last_launches; }
+
+void sparse_attn_trace_enable(int on) {
+  std::lock_guard<std::mutex> lock(g_trace_mu);
+  g_trace_on = on != 0;
+}
+
+int32_t sparse_attn_trace_read(int32_t max, const char** names, double* total_ms,
+                               int32_t* counts) {
+  std::lock_guard<std::mutex> lock(g_trace_mu);
+  std::vector<const char*> nm;
+  std::vector<double> ms;
+  std::vector<int32_t> ct;
+  for (const TraceRec& r : g_trace) {
+    float t = 0.f;
+    cudaEventSynchronize(r.b);
+    cudaEventElapsedTime(&t, r.a, r.b);
+    size_t k = 0;
+    while (k < nm.size() && nm[k] != r.name) ++k;
+    if (k == nm.size()) { nm.push_back(r.name); ms.push_back(0.0); ct.push_back(0); }
+    ms[k] += t;
+    ct[k] += 1;
+    g_ev_pool.push_back(r.a);
+    g_ev_pool.push_back(r.b);
+  }
+  g_trace.clear();
+  for (size_t k = 0; k < nm.size() && (int32_t)k < max; ++k) {
+    if (names) names[k] = nm[k];
+    if (total_ms) total_ms[k] = ms[k];
+    if (counts) counts[k] = ct[k];
+  }
+  return (int32_t)nm.size();
+}
+
+size_t sparse_attn_workspace_size(const sa_params* p, int backward) {
+  sa::Problem pb;
+  if (build_problem(p, &pb) != SA_OK) return 0;
+  if (!backward) return 0;
+  return sa::general_bwd_layout(pb).total;
+}
+
+sa_status sparse_attn_fwd(const sa_params* p, const void* q, const void* k, const void* v,
+                          const float* alpha, void* o, float* lse, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  sa::Problem pb;
+  sa_status s = build_problem(p, &pb);
+  if (s != SA_OK) return s;
+  if (!q || !k || !v || !alpha || !o) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse && !aligned4(lse)) || !aligned4(alpha))
+    return SA_ERR_INVALID_ARG;
+  if (workspace_bytes < sparse_attn_workspace_size(p, 0)) return SA_ERR_WORKSPACE;
+  (void)workspace;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float2* rope = nullptr;
+  if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
+  sa::FwdPtrs a = {q, k, v, alpha, o, lse, rope};
+  int launches = 0;
+  if (sa::launch_fwd_general(pb, a, st, &launches) != cudaSuccess) return SA_ERR_CUDA;
+  g_last_launches = launches;
+  return SA_OK;
+}
+
+sa_status sparse_attn_bwd(const sa_params* p, const void* q, const void* k, const void* v,
+                          const void* o, const float* lse, const void* dout, const float* alpha,
+                          void* dq, void* dk, void* dv, float* dalpha, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  sa::Problem pb;
+  sa_status s = build_problem(p, &pb);
+  if (s != SA_OK) return s;
+  const void* tensors[] = {q, k, v, o, dout, dq, dk, dv};
+  for (const void* x : tensors)
+    if (!x || !aligned16(x)) return SA_ERR_INVALID_ARG;
+  const void* vectors[] = {lse, alpha, dalpha};
+  for (const void* x : vectors)
+    if (!x || !aligned4(x)) return SA_ERR_INVALID_ARG;
+  const size_t need = sparse_attn_workspace_size(p, 1);
+  if (workspace_bytes < need || (need && (!workspace || !aligned16(workspace))))
+    return SA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float2* rope = nullptr;
+  if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
+  sa::BwdPtrs a = {q, k, v, o, dout, lse, alpha, dq, dk, dv, dalpha, rope, workspace};
+  int launches = 0;
+  if (sa::launch_bwd_general(pb, a, st, &launches) != cudaSuccess) return SA_ERR_CUDA;
+  g_last_launches = launches;
+  return SA_OK;
+}
+
+}  // extern "C"

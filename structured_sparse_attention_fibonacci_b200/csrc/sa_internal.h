@@ -1,0 +1,54 @@
+// Internal interface between the C ABI (sa_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "sparse_attn.h"
+
+namespace sa {
+
+// Validated problem description shared by every launcher.
+struct Problem {
+  int L, B, H, T, D, W, n_off, S;
+  float scale;                  // resolved (1/sqrt(D) when the caller passed <= 0)
+  sa_dtype dtype;
+  int f[SA_MAX_OFFSETS];
+  int64_t units() const { return (int64_t)L * B * H; }
+};
+
+struct FwdPtrs {
+  const void* q; const void* k; const void* v;
+  const float* alpha;
+  void* o; float* lse;
+  const float2* rope;           // [T_cap][D/2] (cos, sin)
+};
+
+struct BwdPtrs {
+  const void* q; const void* k; const void* v; const void* o; const void* dout;
+  const float* lse; const float* alpha;
+  void* dq; void* dk; void* dv; float* dalpha;
+  const float2* rope;
+  void* workspace;
+};
+
+// Workspace carving of the general backward (offsets in bytes).
+struct BwdLayout {
+  size_t d_off, dal_off, sink_off, total;
+  int n_qtiles;                 // query tiles per (layer, batch, head) unit
+};
+
+BwdLayout general_bwd_layout(const Problem& pb);
+
+// Tracing hook: brackets one kernel launch with events when tracing is on.
+// Call with begin = true just before the launch and false just after it.
+void trace_mark(const char* kernel, cudaStream_t st, bool begin);
+
+// Each launcher returns the first CUDA error it saw and adds the number of
+// kernels it enqueued to *launches.
+cudaError_t launch_rope_table(float2* tab, int T, int D, double base, cudaStream_t st);
+cudaError_t launch_fwd_general(const Problem& pb, const FwdPtrs& a, cudaStream_t st, int* launches);
+cudaError_t launch_bwd_general(const Problem& pb, const BwdPtrs& a, cudaStream_t st, int* launches);
+
+}  // namespace sa

@@ -1,0 +1,82 @@
+"""Shared helpers for the GPU parity tests: run the CUDA path and the oracle on
+the same seeded inputs and compare with the stated tolerances.
+
+Tolerances (written here, used by every parity test):
+  fp32 inputs : max |GPU - oracle| <= 1e-5 on O, LSE, dQ, dK, dV;
+                |d alpha| relative error <= 1e-5 (it is a sum of many terms).
+  bf16 inputs : max |GPU - oracle| <= 1e-2 on O (stored as bf16) and 1e-3 on
+                LSE (fp32); relative Frobenius norm <= 5e-2 on dQ, dK, dV and
+                relative error <= 5e-2 on d alpha.
+The oracle is the fp64 build, fed the exact values the GPU reads (bf16 inputs
+upcast), so the comparison measures only the GPU path's rounding.
+"""
+import numpy as np
+import torch
+
+import oracle
+import structured_sparse_attention_fibonacci_b200 as sa
+
+TOL = {
+    torch.float32: dict(o_abs=1e-5, lse_abs=1e-5, grad_abs=1e-5, grad_rel=None, dal_rel=1e-5),
+    torch.bfloat16: dict(o_abs=1e-2, lse_abs=1e-3, grad_abs=None, grad_rel=5e-2, dal_rel=5e-2),
+}
+
+
+def rel_norm(a, b):
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def to_np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def run_gpu_fwd(q, k, v, alpha, **kw):
+    o, lse = sa.fwd(q, k, v, alpha, **kw)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+def check_fwd(o_gpu, lse_gpu, o_ref, lse_ref, dtype, what=""):
+    tol = TOL[dtype]
+    o_gpu, lse_gpu = to_np(o_gpu), to_np(lse_gpu)
+    assert np.array_equal(np.isnan(o_gpu), np.isnan(o_ref)), f"{what}: NaN pattern of O"
+    fin = ~np.isnan(o_ref)
+    err_o = np.abs(o_gpu - o_ref)[fin].max(initial=0.0)
+    err_l = np.abs(lse_gpu - lse_ref)[~np.isnan(lse_ref)].max(initial=0.0)
+    assert err_o <= tol["o_abs"], f"{what}: O max abs err {err_o:.3e}"
+    assert err_l <= tol["lse_abs"], f"{what}: LSE max abs err {err_l:.3e}"
+    return err_o, err_l
+
+
+def check_bwd(gpu, ref, dtype, what=""):
+    tol = TOL[dtype]
+    out = {}
+    for name, g, r in zip(("dQ", "dK", "dV"), gpu[:3], ref[:3]):
+        g = to_np(g)
+        assert np.array_equal(np.isnan(g), np.isnan(r)), f"{what}: NaN pattern of {name}"
+        fin = ~np.isnan(r)
+        if tol["grad_abs"] is not None:
+            e = np.abs(g - r)[fin].max(initial=0.0)
+            assert e <= tol["grad_abs"], f"{what}: {name} max abs err {e:.3e}"
+        else:
+            e = rel_norm(g[fin], r[fin])
+            assert e <= tol["grad_rel"], f"{what}: {name} rel-norm err {e:.3e}"
+        out[name] = e
+    dal_g, dal_r = to_np(gpu[3]), np.asarray(ref[3])
+    fin = ~np.isnan(dal_r)
+    assert np.array_equal(np.isnan(dal_g), ~fin), f"{what}: NaN pattern of dalpha"
+    e = np.abs(dal_g - dal_r)[fin] / np.maximum(np.abs(dal_r[fin]), 1e-3)
+    e = float(e.max(initial=0.0))
+    assert e <= tol["dal_rel"], f"{what}: dalpha rel err {e:.3e} ({dal_g} vs {dal_r})"
+    out["dalpha"] = e
+    return out
+
+
+def oracle_fwd(q, k, v, alpha, **kw):
+    return oracle.fwd(to_np(q), to_np(k), to_np(v), to_np(alpha).astype(np.float32), **kw)
+
+
+def oracle_bwd(q, k, v, dout, alpha, **kw):
+    return oracle.bwd(to_np(q), to_np(k), to_np(v), to_np(dout),
+                      to_np(alpha).astype(np.float32), **kw)

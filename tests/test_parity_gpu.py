@@ -1,0 +1,131 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.  Tolerances are in tests/parity.py."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import structured_sparse_attention_fibonacci_b200 as sa
+from structured_sparse_attention_fibonacci_b200.inputs import (FIB15, WORKLOADS, make_dout,
+                                                                make_inputs)
+from parity import check_bwd, check_fwd, oracle_bwd, oracle_fwd, run_gpu_fwd, to_np
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _inputs(shape, dtype, seed, with_dout=True):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    ts = [torch.randn(shape, generator=g, dtype=torch.float32).to(dtype)
+          for _ in range(4 if with_dout else 3)]
+    return [t.to(DEV) for t in ts]
+
+
+# (name, dtype, (L, B, H, T, D), window, sinks, alphas, offsets)
+SMALL = [
+    ("tiny_fp32_cfg", torch.float32, (1, 1, 2, 64, 16), 6, 0, [1.0], FIB15),
+    ("stagger_ragged_bf16", torch.bfloat16, (3, 1, 2, 300, 64), 12, 0, [0.5, 0.9666667, 1.5], FIB15),
+    ("past_987_bf16", torch.bfloat16, (2, 1, 2, 1100, 64), 12, 0, [1.0, 1.1234], FIB15),
+    ("window64_sinks_bf16", torch.bfloat16, (1, 1, 2, 700, 64), 64, 4, [1.0], FIB15),
+    ("d32_fp32", torch.float32, (2, 1, 2, 77, 32), 3, 2, [0.77, 1.33], FIB15),
+    ("d128_fp32", torch.float32, (1, 2, 1, 50, 128), 5, 1, [1.2], FIB15),
+    ("d128_bf16", torch.bfloat16, (1, 1, 2, 90, 128), 7, 3, [0.61], FIB15),
+    ("d16_w1_bf16", torch.bfloat16, (1, 1, 3, 17, 16), 1, 0, [0.93], FIB15),
+    ("t1_fp32", torch.float32, (2, 1, 1, 1, 64), 12, 4, [1.0, 0.5], FIB15),
+    ("t2_fp32", torch.float32, (1, 1, 1, 2, 64), 12, 4, [0.5], FIB15),
+    ("w_ge_t_fp32", torch.float32, (1, 1, 2, 33, 64), 40, 0, [1.0], FIB15),
+    ("no_offsets_fp32", torch.float32, (1, 1, 2, 45, 64), 4, 2, [1.0], ()),
+    ("offsets_beyond_t_fp32", torch.float32, (1, 1, 1, 40, 64), 2, 0, [1.5], FIB15),
+    ("custom_pow2_bf16", torch.bfloat16, (1, 1, 2, 260, 64), 8, 0, [1.0],
+     (1, 2, 4, 8, 16, 32, 64, 128, 256)),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_fwd_bwd_small(case):
+    name, dtype, shape, W, S, alphas, offs = case
+    q, k, v, do = _inputs(shape, dtype, seed=zlib.crc32(name.encode()) % 10000)
+    alpha = torch.tensor(alphas, dtype=torch.float32, device=DEV)
+    kw = dict(window=W, sinks=S, offsets=offs)
+    o, lse = run_gpu_fwd(q, k, v, alpha, **kw)
+    o_ref, lse_ref = oracle_fwd(q, k, v, alpha, **kw)
+    check_fwd(o, lse, o_ref, lse_ref, dtype, name)
+    grads = sa.bwd(q, k, v, o, lse, do, alpha, **kw)
+    torch.cuda.synchronize()
+    ref = oracle_bwd(q, k, v, do, alpha, **kw)
+    check_bwd(grads, ref, dtype, name)
+
+
+def test_nan_alpha_poisons_only_its_layer():
+    q, k, v, do = _inputs((2, 1, 2, 40, 64), torch.float32, seed=3)
+    alpha = torch.tensor([float("nan"), 1.0], device=DEV)
+    o, lse = run_gpu_fwd(q, k, v, alpha, window=4)
+    assert torch.isnan(o[0]).all() and torch.isnan(lse[0]).all()
+    o_ref, lse_ref = oracle_fwd(q, k, v, alpha, window=4)
+    check_fwd(o, lse, o_ref, lse_ref, torch.float32, "nan alpha")
+    grads = sa.bwd(q, k, v, o, lse, do, alpha, window=4)
+    check_bwd(grads, oracle_bwd(q, k, v, do, alpha, window=4), torch.float32, "nan alpha bwd")
+
+
+def test_backward_is_deterministic():
+    q, k, v, do = _inputs((2, 2, 2, 513, 64), torch.bfloat16, seed=11)
+    alpha = torch.tensor([0.71, 1.29], device=DEV)
+    o, lse = run_gpu_fwd(q, k, v, alpha, window=12, sinks=2)
+    a = [t.clone() for t in sa.bwd(q, k, v, o, lse, do, alpha, window=12, sinks=2)]
+    b = sa.bwd(q, k, v, o, lse, do, alpha, window=12, sinks=2)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_streams_are_respected():
+    q, k, v, _ = _inputs((1, 1, 2, 200, 64), torch.bfloat16, seed=12)
+    alpha = torch.tensor([1.1], device=DEV)
+    ref, _ = run_gpu_fwd(q, k, v, alpha, window=12)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o, _ = sa.fwd(q, k, v, alpha, window=12)
+    s.synchronize()
+    assert torch.equal(o, ref)
+
+
+# ---- full-size workloads, the launch the benchmark times; sampled units ------
+
+def _sample_units(wl, n):
+    rng = np.random.default_rng(123)
+    units = {(0, 0, 0), (wl.L - 1, wl.B - 1, wl.H - 1)}
+    while len(units) < min(n, wl.L * wl.B * wl.H):
+        units.add((int(rng.integers(wl.L)), int(rng.integers(wl.B)), int(rng.integers(wl.H))))
+    return sorted(units)
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_full_workload_sampled(name):
+    wl = WORKLOADS[name]
+    ts = make_inputs(wl, device=DEV)
+    q, k, v = ts[:3]
+    alpha = wl.alpha().to(DEV)
+    kw = dict(window=wl.window, sinks=wl.sinks, offsets=wl.offsets, rope_base=wl.rope_base)
+    o, lse = run_gpu_fwd(q, k, v, alpha, **kw)
+    for (l, b, h) in _sample_units(wl, 4):
+        sl = (slice(l, l + 1), slice(b, b + 1), slice(h, h + 1))
+        o_ref, lse_ref = oracle_fwd(q[sl], k[sl], v[sl], alpha[l:l + 1], **kw)
+        check_fwd(o[sl], lse[sl], o_ref, lse_ref, wl.dtype, f"{name} unit {(l, b, h)}")
+    if not wl.backward:
+        return
+    do = ts[3]
+    grads = sa.bwd(q, k, v, o, lse, do, alpha, **kw)
+    torch.cuda.synchronize()
+    for (l, b, h) in _sample_units(wl, 3):
+        sl = (slice(l, l + 1), slice(b, b + 1), slice(h, h + 1))
+        ref = oracle_bwd(q[sl], k[sl], v[sl], do[sl], alpha[l:l + 1], **kw)
+        # d alpha of a single unit is not the layer sum: compare dQ/dK/dV here
+        g = tuple(x[sl] for x in grads[:3]) + (torch.tensor(ref[3]),)
+        check_bwd(g, ref, wl.dtype, f"{name} bwd unit {(l, b, h)}")
+    for l in (0, wl.L - 1):                  # d alpha: the whole layer
+        sl = slice(l, l + 1)
+        ref = oracle_bwd(q[sl], k[sl], v[sl], do[sl], alpha[sl], **kw)
+        e = abs(float(grads[3][l]) - float(ref[3][0])) / max(abs(float(ref[3][0])), 1e-3)
+        assert e <= 5e-2, (l, float(grads[3][l]), float(ref[3][0]))
