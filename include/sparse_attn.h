@@ -136,6 +136,13 @@ const char* sparse_attn_status_string(sa_status s);
 int32_t sparse_attn_last_launch_count(void);
 
 /*
+ * Diagnostics: with on != 0, every later call runs the general kernels (any
+ * dtype and head dim) even where a specialised kernel exists (bf16, D = 64).
+ * Process wide; off by default.  Used to test the two paths against each other.
+ */
+void sparse_attn_force_general(int on);
+
+/*
  * Kernel tracing (diagnostics).  While enabled (on != 0), every kernel the
  * library enqueues is bracketed by two CUDA events recorded on the same
  * stream.  sparse_attn_trace_read waits for all recorded events, writes up to

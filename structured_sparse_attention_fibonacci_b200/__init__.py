@@ -31,7 +31,7 @@ MAX_SINKS = 16
 
 EXPORTED = ("sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_workspace_size",
             "sparse_attn_status_string", "sparse_attn_last_launch_count",
-            "sparse_attn_trace_enable", "sparse_attn_trace_read")
+            "sparse_attn_trace_enable", "sparse_attn_trace_read", "sparse_attn_force_general")
 
 
 class SaParams(ctypes.Structure):
@@ -73,6 +73,8 @@ def lib():
         L.sparse_attn_status_string.argtypes = [ctypes.c_int]
         L.sparse_attn_last_launch_count.restype = ctypes.c_int32
         L.sparse_attn_last_launch_count.argtypes = []
+        L.sparse_attn_force_general.restype = None
+        L.sparse_attn_force_general.argtypes = [ctypes.c_int]
         L.sparse_attn_trace_enable.restype = None
         L.sparse_attn_trace_enable.argtypes = [ctypes.c_int]
         L.sparse_attn_trace_read.restype = ctypes.c_int32
@@ -116,6 +118,11 @@ def workspace_size(shape, dtype, *, backward, **kw) -> int:
 def last_launch_count() -> int:
     """Kernels enqueued by the latest fwd/bwd call on this thread."""
     return int(lib().sparse_attn_last_launch_count())
+
+
+def force_general(on: bool = True) -> None:
+    """Route every call through the general kernels (diagnostics / testing)."""
+    lib().sparse_attn_force_general(int(bool(on)))
 
 
 def trace_enable(on: bool = True) -> None:

@@ -13,6 +13,7 @@
 namespace {
 
 thread_local int32_t g_last_launches = 0;
+int g_force_general = 0;  // diagnostics: route every call through the general kernels
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -135,6 +136,8 @@ const char* sparse_attn_status_string(sa_status s) {
 
 int32_t sparse_attn_last_launch_count(void) { return g_last_launches; }
 
+void sparse_attn_force_general(int on) { g_force_general = on != 0; }
+
 void sparse_attn_trace_enable(int on) {
   std::lock_guard<std::mutex> lock(g_trace_mu);
   g_trace_on = on != 0;
@@ -191,7 +194,10 @@ sa_status sparse_attn_fwd(const sa_params* p, const void* q, const void* k, cons
   if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
   sa::FwdPtrs a = {q, k, v, alpha, o, lse, rope};
   int launches = 0;
-  if (sa::launch_fwd_general(pb, a, st, &launches) != cudaSuccess) return SA_ERR_CUDA;
+  cudaError_t e = (!g_force_general && sa::fast_fwd_supported(pb))
+                      ? sa::launch_fwd_fast(pb, a, st, &launches)
+                      : sa::launch_fwd_general(pb, a, st, &launches);
+  if (e != cudaSuccess) return SA_ERR_CUDA;
   g_last_launches = launches;
   return SA_OK;
 }

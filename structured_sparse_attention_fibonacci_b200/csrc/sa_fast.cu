@@ -1,0 +1,493 @@
+// Staged forward for bf16 inputs with head dim 64 (the shape of every bf16
+// workload of "Depth-Staggered Fibonacci Spacing for Sparse Attention":
+// hidden 512 = 8 heads x 64, technical summary, Methodology).
+//
+// One CTA owns a tile of M consecutive queries of one (layer, batch, head).
+//  * Lane mapping: a group of 4 lanes owns 4 consecutive queries; lane c of
+//    the group holds dims [8c, 8c+8) and [32+8c, 32+8c+8) of each (a rotate-
+//    half RoPE pair stays in one lane).  Every staged row chunk a lane reads
+//    is reused for up to 4 queries (window) or 2 queries (an interpolated
+//    offset), which keeps shared-memory traffic near one byte per FMA.
+//  * Partial dot products of the 4 lanes are combined by a 4-lane transpose
+//    reduce-scatter, after which each lane owns one query's full scores.
+//  * Staging: the tile's members are visited in increasing lag order (window,
+//    then the offsets sorted by f).  Each member needs a contiguous row range;
+//    only rows below everything staged so far are fetched, into a ring of
+//    shared-memory rows, so every row of the tile's union is read from L2 once
+//    per pass.  K rows are rotated (RoPE) on the way in; rows are stored as
+//    bf16 with a 16-byte-chunk XOR swizzle.
+//  * An offset whose rows lie inside the window ("near") costs nothing: its
+//    score is the interpolation of two window scores, and its probability is
+//    folded into the two window weights used for PV.
+//  * Two passes over the members: scores (K ring), softmax by the owner lane,
+//    then PV (V ring).
+#include <algorithm>
+
+#include "sa_device.cuh"
+#include "sa_internal.h"
+
+namespace sa {
+
+namespace {
+
+constexpr int kD = 64;
+constexpr int kChunks = 8;             // 16-byte chunks per bf16 row
+constexpr int kFastM = 128;            // queries per CTA = threads per CTA
+
+struct FastArgs {
+  int B, H, T, W, n_off, S, n_tiles;
+  int ring_rows, sc_stride;
+  float scale;
+  int f[SA_MAX_OFFSETS];               // ascending
+  const __nv_bfloat16* q; const __nv_bfloat16* k; const __nv_bfloat16* v;
+  const float* alpha; const float2* rope;
+  __nv_bfloat16* o; float* lse;
+};
+
+__device__ __forceinline__ void unpack8(const uint4 u, float* x) {
+  x[0] = bf16lo(u.x); x[1] = bf16hi(u.x); x[2] = bf16lo(u.y); x[3] = bf16hi(u.y);
+  x[4] = bf16lo(u.z); x[5] = bf16hi(u.z); x[6] = bf16lo(u.w); x[7] = bf16hi(u.w);
+}
+
+__device__ __forceinline__ uint4 pack8(const float* x) {
+  return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                    pack_bf16x2(x[6], x[7]));
+}
+
+__device__ __forceinline__ int swz(int slot) { return (slot >> 2) & 7; }
+
+// This lane's 16 dims of ring slot `slot`.
+__device__ __forceinline__ void ring_load(const uint4* ring, int slot, int c, float (&x)[16]) {
+  const int s = swz(slot);
+  unpack8(ring[slot * kChunks + (c ^ s)], x);
+  unpack8(ring[slot * kChunks + ((c + 4) ^ s)], x + 8);
+}
+
+__device__ __forceinline__ float dot16(const float (&q)[16], const float (&x)[16]) {
+  float a = 0.f, b = 0.f;
+#pragma unroll
+  for (int h = 0; h < 16; h += 2) {
+    a = fmaf(q[h], x[h], a);
+    b = fmaf(q[h + 1], x[h + 1], b);
+  }
+  return a + b;
+}
+
+__device__ __forceinline__ void axpy16(float (&o)[16], float p, const float (&x)[16]) {
+#pragma unroll
+  for (int h = 0; h < 16; ++h) o[h] = fmaf(p, x[h], o[h]);
+}
+
+// p[q][l] are partial sums held by the 4 lanes of a group (lane c = 2*hi+lo);
+// out[l] receives the sum over the 4 lanes of p[c][l].
+template <int L>
+__device__ __forceinline__ void reduce_scatter4(const float (&p)[4][L], float (&out)[L], int c) {
+  const bool hi = (c >> 1) & 1, lo = c & 1;
+  float r[2][L];
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+#pragma unroll
+    for (int l = 0; l < L; ++l) {
+      const float keep = hi ? p[2 + j][l] : p[j][l];
+      const float send = hi ? p[j][l] : p[2 + j][l];
+      r[j][l] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+#pragma unroll
+  for (int l = 0; l < L; ++l) {
+    const float keep = lo ? r[1][l] : r[0][l];
+    const float send = lo ? r[0][l] : r[1][l];
+    out[l] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+  }
+}
+
+// Stage rows [a, b) of src (bf16 [T][64]) into ring slots row % ring_rows,
+// rotating K rows by RoPE at their own position.  One task = one row and one
+// RoPE pair-chunk p (dims [8p, 8p+8) and [32+8p, 32+8p+8)).
+template <bool ROT>
+__device__ __forceinline__ void stage_rows(uint4* ring, int ring_rows, const __nv_bfloat16* src,
+                                           const float2* rope, int a, int b) {
+  const int n = (b - a) * 4;
+  for (int task = threadIdx.x; task < n; task += blockDim.x) {
+    const int row = a + (task >> 2), p = task & 3;
+    const uint4* g = reinterpret_cast<const uint4*>(src + (size_t)row * kD);
+    uint4 u0 = __ldg(g + p), u1 = __ldg(g + p + 4);
+    if (ROT) {
+      float x1[8], x2[8];
+      unpack8(u0, x1);
+      unpack8(u1, x2);
+      const float4* cs = reinterpret_cast<const float4*>(rope + (size_t)row * 32 + 8 * p);
+#pragma unroll
+      for (int h = 0; h < 8; h += 2) {
+        const float4 t = __ldg(cs + h / 2);
+        float a0 = x1[h], b0 = x2[h], a1 = x1[h + 1], b1 = x2[h + 1];
+        x1[h] = a0 * t.x - b0 * t.y;  x2[h] = b0 * t.x + a0 * t.y;
+        x1[h + 1] = a1 * t.z - b1 * t.w;  x2[h + 1] = b1 * t.z + a1 * t.w;
+      }
+      u0 = pack8(x1);
+      u1 = pack8(x2);
+    }
+    const int slot = row % ring_rows;
+    const int s = swz(slot);
+    ring[slot * kChunks + (p ^ s)] = u0;
+    ring[slot * kChunks + ((p + 4) ^ s)] = u1;
+  }
+}
+
+// Sink rows 0..S-1 into a plain (unswizzled) buffer.
+template <bool ROT>
+__device__ __forceinline__ void stage_sinks(uint4* buf, int S, const __nv_bfloat16* src,
+                                            const float2* rope) {
+  for (int task = threadIdx.x; task < S * 4; task += blockDim.x) {
+    const int row = task >> 2, p = task & 3;
+    const uint4* g = reinterpret_cast<const uint4*>(src + (size_t)row * kD);
+    uint4 u0 = __ldg(g + p), u1 = __ldg(g + p + 4);
+    if (ROT) {
+      float x1[8], x2[8];
+      unpack8(u0, x1);
+      unpack8(u1, x2);
+      const float4* cs = reinterpret_cast<const float4*>(rope + (size_t)row * 32 + 8 * p);
+#pragma unroll
+      for (int h = 0; h < 8; h += 2) {
+        const float4 t = __ldg(cs + h / 2);
+        float a0 = x1[h], b0 = x2[h], a1 = x1[h + 1], b1 = x2[h + 1];
+        x1[h] = a0 * t.x - b0 * t.y;  x2[h] = b0 * t.x + a0 * t.y;
+        x1[h + 1] = a1 * t.z - b1 * t.w;  x2[h + 1] = b1 * t.z + a1 * t.w;
+      }
+      u0 = pack8(x1);
+      u1 = pack8(x2);
+    }
+    buf[row * kChunks + p] = u0;
+    buf[row * kChunks + p + 4] = u1;
+  }
+}
+
+__device__ __forceinline__ void sink_load(const uint4* buf, int s, int c, float (&x)[16]) {
+  unpack8(buf[s * kChunks + c], x);
+  unpack8(buf[s * kChunks + c + 4], x + 8);
+}
+
+// Window scores for lags [d0, d0 + LC): rows ig+3-d0-u, u = 0..LC+2; query q
+// (row ig+q) takes row u at lag d0 + (q + u - 3).
+template <int LC>
+__device__ __forceinline__ void window_scores(const uint4* ring, int ring_rows, int ig, int d0,
+                                              int c, const float (&q)[4][16], float* sc_row) {
+  float acc[4][LC];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int l = 0; l < LC; ++l) acc[a][l] = 0.f;
+#pragma unroll
+  for (int u = 0; u < LC + 3; ++u) {
+    const int row = max(ig + 3 - d0 - u, 0);
+    float x[16];
+    ring_load(ring, row % ring_rows, c, x);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int l = a + u - 3;
+      if (l >= 0 && l < LC) acc[a][l] += dot16(q[a], x);
+    }
+  }
+  float out[LC];
+  reduce_scatter4<LC>(acc, out, c);
+#pragma unroll
+  for (int l = 0; l < LC; ++l) sc_row[d0 + l] = out[l];
+}
+
+// Window PV for lags [d0, d0 + LC) with weights sc[query][lag].
+template <int LC>
+__device__ __forceinline__ void window_pv(const uint4* ring, int ring_rows, int ig, int d0, int c,
+                                          const float* sc, int stride, float (&o)[4][16]) {
+  float pw[4][LC];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int l = 0; l < LC; ++l) pw[a][l] = sc[a * stride + d0 + l];
+#pragma unroll
+  for (int u = 0; u < LC + 3; ++u) {
+    const int row = max(ig + 3 - d0 - u, 0);
+    float x[16];
+    ring_load(ring, row % ring_rows, c, x);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int l = a + u - 3;
+      if (l >= 0 && l < LC) axpy16(o[a], pw[a][l], x);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
+  constexpr int M = kFastM;
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint4* ring = reinterpret_cast<uint4*>(smem);
+  uint4* sinkb = ring + (size_t)a.ring_rows * kChunks;
+  float* sc = reinterpret_cast<float*>(sinkb + (size_t)a.S * kChunks);
+  __shared__ OffGeo sg[SA_MAX_OFFSETS];
+  __shared__ int s_fold[SA_MAX_OFFSETS];
+
+  const int unit = blockIdx.x / a.n_tiles, tile = blockIdx.x % a.n_tiles;
+  const int layer = unit / (a.B * a.H);
+  const int T = a.T, W = a.W, S = a.S, n_off = a.n_off;
+  const int i0 = tile * M;
+  const int t = threadIdx.x, gid = t >> 2, c = t & 3;
+  const int ig = i0 + 4 * gid;
+  const size_t ub = (size_t)unit * T * kD;
+  const __nv_bfloat16* Q = a.q + ub;
+  const __nv_bfloat16* K = a.k + ub;
+  const __nv_bfloat16* V = a.v + ub;
+
+  int bad = 0;
+  if (t < n_off) {
+    const OffGeo g = offset_geometry(__ldg(a.alpha + layer), a.f[t]);
+    sg[t] = g;
+    bad = !g.ok;
+    s_fold[t] = g.ok && (g.lo + (g.w != 0.f ? 1 : 0) <= W - 1);
+  }
+  bad = __syncthreads_or(bad);
+  if (bad) {  // the layer has an offset with no defined row: NaN outputs
+    const float qnan = __int_as_float(0x7fc00000);
+    for (int e = t; e < M * kChunks; e += M) {
+      const int i = i0 + e / kChunks;
+      if (i < T) {
+        float x[8];
+#pragma unroll
+        for (int h = 0; h < 8; ++h) x[h] = qnan;
+        reinterpret_cast<uint4*>(a.o + ub + (size_t)i * kD)[e % kChunks] = pack8(x);
+        if (e % kChunks == 0 && a.lse) a.lse[(size_t)unit * T + i] = qnan;
+      }
+    }
+    return;
+  }
+
+  // zero the ring and the sink rows so unstaged slots always hold finite values
+  // (sink rows s >= T are never attended and never staged)
+  for (int e = t; e < (a.ring_rows + S) * kChunks; e += M) ring[e] = make_uint4(0, 0, 0, 0);
+  const int S_rows = min(S, T);
+
+  // this lane's slice of its 4 queries, rotated and scaled
+  float q[4][16];
+#pragma unroll
+  for (int qq = 0; qq < 4; ++qq) {
+    const int row = min(ig + qq, T - 1);
+    const uint4* g = reinterpret_cast<const uint4*>(Q + (size_t)row * kD);
+    float x1[8], x2[8];
+    unpack8(__ldg(g + c), x1);
+    unpack8(__ldg(g + c + 4), x2);
+    const float4* cs = reinterpret_cast<const float4*>(a.rope + (size_t)row * 32 + 8 * c);
+#pragma unroll
+    for (int h = 0; h < 8; h += 2) {
+      const float4 tt = __ldg(cs + h / 2);
+      q[qq][h] = (x1[h] * tt.x - x2[h] * tt.y) * a.scale;
+      q[qq][h + 8] = (x2[h] * tt.x + x1[h] * tt.y) * a.scale;
+      q[qq][h + 1] = (x1[h + 1] * tt.z - x2[h + 1] * tt.w) * a.scale;
+      q[qq][h + 9] = (x2[h + 1] * tt.z + x1[h + 1] * tt.w) * a.scale;
+    }
+  }
+
+  const int lr = 4 * gid + c;                  // this lane's query, tile-local
+  float* my_sc = sc + (size_t)lr * a.sc_stride;
+  const int win_lo = max(0, i0 - W + 1), win_hi = min(T, i0 + M);
+  const int RB = a.ring_rows;
+
+  // ---------------- pass 1: scores ----------------
+  __syncthreads();
+  stage_rows<true>(ring, RB, K, a.rope, win_lo, win_hi);
+  stage_sinks<true>(sinkb, S_rows, K, a.rope);
+  __syncthreads();
+  {
+    int d0 = 0;
+    while (W - d0 >= 8) { window_scores<8>(ring, RB, ig, d0, c, q, my_sc); d0 += 8; }
+    if (W - d0 >= 4) { window_scores<4>(ring, RB, ig, d0, c, q, my_sc); d0 += 4; }
+    if (W - d0 >= 2) { window_scores<2>(ring, RB, ig, d0, c, q, my_sc); d0 += 2; }
+    if (W - d0 >= 1) { window_scores<1>(ring, RB, ig, d0, c, q, my_sc); d0 += 1; }
+  }
+  for (int s0 = 0; s0 < S; s0 += 4) {
+    float acc[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float x[16];
+      sink_load(sinkb, min(s0 + j, S - 1), c, x);
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) acc[qq][j] = dot16(q[qq], x);
+    }
+    float out[4];
+    reduce_scatter4<4>(acc, out, c);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (s0 + j < S) my_sc[W + s0 + j] = out[j];
+  }
+  int low = win_lo;
+  for (int kk = 0; kk < n_off; ++kk) {
+    if (s_fold[kk]) continue;                  // CTA-uniform
+    const OffGeo g = sg[kk];
+    const int two = g.w != 0.f;
+    const int seg_lo = max(0, i0 - g.lo - two), seg_hi = min(T, i0 + M - g.lo);
+    if (seg_lo < low && seg_lo < seg_hi) {
+      __syncthreads();
+      stage_rows<true>(ring, RB, K, a.rope, seg_lo, min(seg_hi, low));
+      low = seg_lo;
+      __syncthreads();
+    }
+    float pa[4] = {0.f, 0.f, 0.f, 0.f}, pb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 5; ++u) {
+      if (u == 0 && !two) continue;
+      const int row = max(ig - g.lo - 1 + u, 0);
+      float x[16];
+      ring_load(ring, row % RB, c, x);
+      if (u <= 3) pb[u] = dot16(q[u], x);
+      if (u >= 1) pa[u - 1] = dot16(q[u - 1], x);
+    }
+    float part[4][1];
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) part[qq][0] = g.wa * pa[qq] + g.w * pb[qq];
+    float out[1];
+    reduce_scatter4<1>(part, out, c);
+    my_sc[W + S + kk] = out[0];
+  }
+  __syncthreads();
+
+  // ---------------- softmax (owner lane of each query) ----------------
+  {
+    const int i = ig + c;
+    if (i < T) {
+      for (int kk = 0; kk < n_off; ++kk) {
+        if (!s_fold[kk]) continue;
+        const OffGeo g = sg[kk];
+        float s = g.wa * my_sc[g.lo];
+        if (g.w != 0.f) s += g.w * my_sc[g.lo + 1];
+        my_sc[W + S + kk] = s;
+      }
+      float m = -INFINITY;
+      for (int d = 0; d < W; ++d) if (i - d >= 0) m = fmaxf(m, my_sc[d]);
+      for (int s = 0; s < S; ++s) if (s <= i) m = fmaxf(m, my_sc[W + s]);
+      for (int kk = 0; kk < n_off; ++kk) if (i - sg[kk].c >= 0) m = fmaxf(m, my_sc[W + S + kk]);
+      float l = 0.f;
+      for (int d = 0; d < W; ++d) {
+        const float p = (i - d >= 0) ? __expf(my_sc[d] - m) : 0.f;
+        my_sc[d] = p; l += p;
+      }
+      for (int s = 0; s < S; ++s) {
+        const float p = (s <= i) ? __expf(my_sc[W + s] - m) : 0.f;
+        my_sc[W + s] = p; l += p;
+      }
+      for (int kk = 0; kk < n_off; ++kk) {
+        const float p = (i - sg[kk].c >= 0) ? __expf(my_sc[W + S + kk] - m) : 0.f;
+        my_sc[W + S + kk] = p; l += p;
+      }
+      const float inv = 1.f / l;
+      for (int d = 0; d < W + S + n_off; ++d) my_sc[d] *= inv;
+      for (int kk = 0; kk < n_off; ++kk) {     // fold near offsets into window weights
+        if (!s_fold[kk]) continue;
+        const OffGeo g = sg[kk];
+        const float p = my_sc[W + S + kk];
+        my_sc[g.lo] += g.wa * p;
+        if (g.w != 0.f) my_sc[g.lo + 1] += g.w * p;
+      }
+      if (a.lse) a.lse[(size_t)unit * T + i] = m + __logf(l);
+    } else {
+      for (int d = 0; d < W + S + n_off; ++d) my_sc[d] = 0.f;
+    }
+  }
+  __syncthreads();
+
+  // ---------------- pass 2: PV ----------------
+  float o[4][16];
+#pragma unroll
+  for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+    for (int h = 0; h < 16; ++h) o[qq][h] = 0.f;
+  const float* grp_sc = sc + (size_t)(4 * gid) * a.sc_stride;
+  stage_rows<false>(ring, RB, V, a.rope, win_lo, win_hi);
+  stage_sinks<false>(sinkb, S_rows, V, a.rope);
+  __syncthreads();
+  {
+    int d0 = 0;
+    while (W - d0 >= 8) { window_pv<8>(ring, RB, ig, d0, c, grp_sc, a.sc_stride, o); d0 += 8; }
+    if (W - d0 >= 4) { window_pv<4>(ring, RB, ig, d0, c, grp_sc, a.sc_stride, o); d0 += 4; }
+    if (W - d0 >= 2) { window_pv<2>(ring, RB, ig, d0, c, grp_sc, a.sc_stride, o); d0 += 2; }
+    if (W - d0 >= 1) { window_pv<1>(ring, RB, ig, d0, c, grp_sc, a.sc_stride, o); d0 += 1; }
+  }
+  for (int s = 0; s < S; ++s) {
+    float x[16];
+    sink_load(sinkb, s, c, x);
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) axpy16(o[qq], grp_sc[qq * a.sc_stride + W + s], x);
+  }
+  low = win_lo;
+  for (int kk = 0; kk < n_off; ++kk) {
+    if (s_fold[kk]) continue;
+    const OffGeo g = sg[kk];
+    const int two = g.w != 0.f;
+    const int seg_lo = max(0, i0 - g.lo - two), seg_hi = min(T, i0 + M - g.lo);
+    if (seg_lo < low && seg_lo < seg_hi) {
+      __syncthreads();
+      stage_rows<false>(ring, RB, V, a.rope, seg_lo, min(seg_hi, low));
+      low = seg_lo;
+      __syncthreads();
+    }
+    float p[4];
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) p[qq] = grp_sc[qq * a.sc_stride + W + S + kk];
+#pragma unroll
+    for (int u = 0; u < 5; ++u) {
+      if (u == 0 && !two) continue;
+      const int row = max(ig - g.lo - 1 + u, 0);
+      float x[16];
+      ring_load(ring, row % RB, c, x);
+      if (u <= 3 && two) axpy16(o[u], p[u] * g.w, x);
+      if (u >= 1) axpy16(o[u - 1], p[u - 1] * g.wa, x);
+    }
+  }
+
+#pragma unroll
+  for (int qq = 0; qq < 4; ++qq) {
+    const int i = ig + qq;
+    if (i < T) {
+      uint4* dst = reinterpret_cast<uint4*>(a.o + ub + (size_t)i * kD);
+      dst[c] = pack8(o[qq]);
+      dst[c + 4] = pack8(o[qq] + 8);
+    }
+  }
+}
+
+}  // namespace
+
+bool fast_fwd_supported(const Problem& pb) {
+  return pb.dtype == SA_DTYPE_BF16 && pb.D == kD && pb.W <= 256;
+}
+
+size_t fast_fwd_smem(const Problem& pb, int* ring_rows, int* sc_stride) {
+  const int rr = ((std::max(kFastM + pb.W - 1, kFastM + 2) + 31) / 32) * 32;
+  const int n_slot = pb.W + pb.S + pb.n_off;
+  const int st = ((n_slot + 3) / 4) * 4 + 4;
+  if (ring_rows) *ring_rows = rr;
+  if (sc_stride) *sc_stride = st;
+  return (size_t)rr * 128 + (size_t)pb.S * 128 + (size_t)kFastM * st * sizeof(float);
+}
+
+cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& p, cudaStream_t st, int* launches) {
+  FastArgs a = {};
+  a.B = pb.B; a.H = pb.H; a.T = pb.T; a.W = pb.W; a.n_off = pb.n_off; a.S = pb.S;
+  a.n_tiles = (pb.T + kFastM - 1) / kFastM;
+  a.scale = pb.scale;
+  for (int k = 0; k < pb.n_off; ++k) a.f[k] = pb.f[k];
+  std::sort(a.f, a.f + pb.n_off);
+  const size_t smem = fast_fwd_smem(pb, &a.ring_rows, &a.sc_stride);
+  a.q = reinterpret_cast<const __nv_bfloat16*>(p.q);
+  a.k = reinterpret_cast<const __nv_bfloat16*>(p.k);
+  a.v = reinterpret_cast<const __nv_bfloat16*>(p.v);
+  a.alpha = p.alpha; a.rope = p.rope;
+  a.o = reinterpret_cast<__nv_bfloat16*>(p.o); a.lse = p.lse;
+  cudaError_t e = cudaFuncSetAttribute(k_fwd_fast, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)((long long)pb.units() * a.n_tiles);
+  trace_mark("fwd_fast", st, true);
+  k_fwd_fast<<<grid, kFastM, smem, st>>>(a);
+  trace_mark("fwd_fast", st, false);
+  e = cudaGetLastError();
+  if (e == cudaSuccess) *launches += 1;
+  return e;
+}
+
+}  // namespace sa

@@ -47,6 +47,11 @@ void trace_mark(const char* kernel, cudaStream_t st, bool begin);
 
 // Each launcher returns the first CUDA error it saw and adds the number of
 // kernels it enqueued to *launches.
+// Staged bf16 / D=64 forward (sa_fast.cu).
+bool fast_fwd_supported(const Problem& pb);
+size_t fast_fwd_smem(const Problem& pb, int* ring_rows, int* sc_stride);
+cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& a, cudaStream_t st, int* launches);
+
 cudaError_t launch_rope_table(float2* tab, int T, int D, double base, cudaStream_t st);
 cudaError_t launch_fwd_general(const Problem& pb, const FwdPtrs& a, cudaStream_t st, int* launches);
 cudaError_t launch_bwd_general(const Problem& pb, const BwdPtrs& a, cudaStream_t st, int* launches);

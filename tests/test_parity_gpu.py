@@ -129,3 +129,51 @@ def test_full_workload_sampled(name):
         ref = oracle_bwd(q[sl], k[sl], v[sl], do[sl], alpha[sl], **kw)
         e = abs(float(grads[3][l]) - float(ref[3][0])) / max(abs(float(ref[3][0])), 1e-3)
         assert e <= 5e-2, (l, float(grads[3][l]), float(ref[3][0]))
+
+
+# ---- the staged bf16 d=64 forward and the general kernels on the same inputs ----
+FAST = [
+    ("fast_tail_129", (2, 1, 2, 129, 64), 12, 0, [0.5, 1.5], FIB15),
+    ("fast_t257_sinks", (1, 2, 1, 257, 64), 12, 4, [1.1], FIB15),
+    ("fast_t1", (1, 1, 2, 1, 64), 12, 4, [1.0], FIB15),
+    ("fast_t3_s16", (1, 1, 1, 3, 64), 2, 16, [0.7], FIB15),
+    ("fast_w64_s16", (1, 1, 2, 600, 64), 64, 16, [1.0], FIB15),
+    ("fast_unsorted_dups", (1, 1, 2, 400, 64), 5, 1, [0.83], (34, 1, 5, 5, 233, 2, 89, 13)),
+    ("fast_alpha0", (1, 1, 1, 70, 64), 3, 0, [0.0], FIB15),
+    ("fast_w1", (1, 1, 2, 200, 64), 1, 0, [1.37], FIB15),
+    ("fast_w7_odd", (2, 1, 1, 300, 64), 7, 3, [0.61, 1.44], FIB15),
+    ("fast_long_1500", (1, 1, 1, 1700, 64), 12, 0, [1.5], FIB15),
+]
+
+
+@pytest.mark.parametrize("case", FAST, ids=[c[0] for c in FAST])
+def test_fast_and_general_forward(case):
+    name, shape, W, S, alphas, offs = case
+    q, k, v, _ = _inputs(shape, torch.bfloat16, seed=zlib.crc32(name.encode()) % 10000)
+    alpha = torch.tensor(alphas, dtype=torch.float32, device=DEV)
+    kw = dict(window=W, sinks=S, offsets=offs)
+    o_ref, lse_ref = oracle_fwd(q, k, v, alpha, **kw)
+    o_fast, lse_fast = run_gpu_fwd(q, k, v, alpha, **kw)
+    check_fwd(o_fast, lse_fast, o_ref, lse_ref, torch.bfloat16, name + " (staged)")
+    sa.force_general(True)
+    try:
+        o_gen, lse_gen = run_gpu_fwd(q, k, v, alpha, **kw)
+    finally:
+        sa.force_general(False)
+    check_fwd(o_gen, lse_gen, o_ref, lse_ref, torch.bfloat16, name + " (general)")
+    # the two paths differ only by fp32 summation order and the bf16 rounding
+    # of the staged rotated keys
+    assert (o_fast.float() - o_gen.float()).abs().max().item() <= 1e-2
+    assert (lse_fast - lse_gen).abs().max().item() <= 1e-2
+
+
+def test_fast_path_is_the_one_dispatched():
+    q, k, v, _ = _inputs((1, 1, 1, 300, 64), torch.bfloat16, seed=5)
+    alpha = torch.tensor([1.0], device=DEV)
+    sa.trace_enable(True)
+    try:
+        run_gpu_fwd(q, k, v, alpha, window=12)
+        names = set(sa.trace_read())
+    finally:
+        sa.trace_enable(False)
+    assert names == {"fwd_fast"}, names
