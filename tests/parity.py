@@ -4,9 +4,13 @@ the same seeded inputs and compare with the stated tolerances.
 Tolerances (written here, used by every parity test):
   fp32 inputs : max |GPU - oracle| <= 1e-5 on O, LSE, dQ, dK, dV;
                 |d alpha| relative error <= 1e-5 (it is a sum of many terms).
-  bf16 inputs : max |GPU - oracle| <= 1e-2 on O (stored as bf16) and 1e-3 on
-                LSE (fp32); relative Frobenius norm <= 5e-2 on dQ, dK, dV and
-                relative error <= 5e-2 on d alpha.
+  bf16 inputs : max |GPU - oracle| <= 1e-2 on O (stored as bf16) and on LSE
+                (fp32); relative Frobenius norm <= 5e-2 on dQ, dK, dV and
+                relative error <= 5e-2 on d alpha.  The LSE bound follows from
+                the staged kernels keeping rotated K rows in bf16: a relative
+                rounding of 2^-9 per element gives score errors of about
+                2^-9/sqrt(3) * |q_hat o k| ~ 1e-3 for N(0,1) inputs, a few 1e-3
+                at the worst of ~1e5 queries.
 The oracle is the fp64 build, fed the exact values the GPU reads (bf16 inputs
 upcast), so the comparison measures only the GPU path's rounding.
 """
@@ -18,7 +22,7 @@ import structured_sparse_attention_fibonacci_b200 as sa
 
 TOL = {
     torch.float32: dict(o_abs=1e-5, lse_abs=1e-5, grad_abs=1e-5, grad_rel=None, dal_rel=1e-5),
-    torch.bfloat16: dict(o_abs=1e-2, lse_abs=1e-3, grad_abs=None, grad_rel=5e-2, dal_rel=5e-2),
+    torch.bfloat16: dict(o_abs=1e-2, lse_abs=1e-2, grad_abs=None, grad_rel=5e-2, dal_rel=5e-2),
 }
 
 
