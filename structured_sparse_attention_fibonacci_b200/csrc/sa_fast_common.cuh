@@ -1,0 +1,140 @@
+// Building blocks of the staged bf16 / head-dim-64 kernels (forward and
+// backward): the row ring in shared memory, its loads and stores, the 16-dim
+// lane slices and the 4-lane reduce-scatter.  See sa_fast.cu for the layout.
+#pragma once
+
+#include "sa_device.cuh"
+#include "sa_internal.h"
+
+namespace sa {
+namespace fast {
+
+constexpr int kD = 64;
+constexpr int kChunks = 8;             // 16-byte chunks per bf16 row
+constexpr int kFastM = 128;            // rows (queries or keys) per CTA = threads per CTA
+
+
+__device__ __forceinline__ void unpack8(const uint4 u, float* x) {
+  x[0] = bf16lo(u.x); x[1] = bf16hi(u.x); x[2] = bf16lo(u.y); x[3] = bf16hi(u.y);
+  x[4] = bf16lo(u.z); x[5] = bf16hi(u.z); x[6] = bf16lo(u.w); x[7] = bf16hi(u.w);
+}
+
+__device__ __forceinline__ uint4 pack8(const float* x) {
+  return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                    pack_bf16x2(x[6], x[7]));
+}
+
+__device__ __forceinline__ int swz(int slot) { return (slot >> 2) & 7; }
+
+// This lane's 16 dims of ring slot `slot`.
+__device__ __forceinline__ void ring_load(const uint4* ring, int slot, int c, float (&x)[16]) {
+  const int s = swz(slot);
+  unpack8(ring[slot * kChunks + (c ^ s)], x);
+  unpack8(ring[slot * kChunks + ((c + 4) ^ s)], x + 8);
+}
+
+__device__ __forceinline__ float dot16(const float (&q)[16], const float (&x)[16]) {
+  float a = 0.f, b = 0.f;
+#pragma unroll
+  for (int h = 0; h < 16; h += 2) {
+    a = fmaf(q[h], x[h], a);
+    b = fmaf(q[h + 1], x[h + 1], b);
+  }
+  return a + b;
+}
+
+__device__ __forceinline__ void axpy16(float (&o)[16], float p, const float (&x)[16]) {
+#pragma unroll
+  for (int h = 0; h < 16; ++h) o[h] = fmaf(p, x[h], o[h]);
+}
+
+// p[q][l] are partial sums held by the 4 lanes of a group (lane c = 2*hi+lo);
+// out[l] receives the sum over the 4 lanes of p[c][l].
+template <int L>
+__device__ __forceinline__ void reduce_scatter4(const float (&p)[4][L], float (&out)[L], int c) {
+  const bool hi = (c >> 1) & 1, lo = c & 1;
+  float r[2][L];
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+#pragma unroll
+    for (int l = 0; l < L; ++l) {
+      const float keep = hi ? p[2 + j][l] : p[j][l];
+      const float send = hi ? p[j][l] : p[2 + j][l];
+      r[j][l] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+#pragma unroll
+  for (int l = 0; l < L; ++l) {
+    const float keep = lo ? r[1][l] : r[0][l];
+    const float send = lo ? r[0][l] : r[1][l];
+    out[l] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+  }
+}
+
+// Stage rows [a, b) of src (bf16 [T][64]) into ring slots row % ring_rows,
+// rotating K rows by RoPE at their own position.  One task = one row and one
+// RoPE pair-chunk p (dims [8p, 8p+8) and [32+8p, 32+8p+8)).
+template <bool ROT>
+__device__ __forceinline__ void stage_rows(uint4* ring, int ring_rows, const __nv_bfloat16* src,
+                                           const float2* rope, int a, int b) {
+  const int n = (b - a) * 4;
+  for (int task = threadIdx.x; task < n; task += blockDim.x) {
+    const int row = a + (task >> 2), p = task & 3;
+    const uint4* g = reinterpret_cast<const uint4*>(src + (size_t)row * kD);
+    uint4 u0 = __ldg(g + p), u1 = __ldg(g + p + 4);
+    if (ROT) {
+      float x1[8], x2[8];
+      unpack8(u0, x1);
+      unpack8(u1, x2);
+      const float4* cs = reinterpret_cast<const float4*>(rope + (size_t)row * 32 + 8 * p);
+#pragma unroll
+      for (int h = 0; h < 8; h += 2) {
+        const float4 t = __ldg(cs + h / 2);
+        float a0 = x1[h], b0 = x2[h], a1 = x1[h + 1], b1 = x2[h + 1];
+        x1[h] = a0 * t.x - b0 * t.y;  x2[h] = b0 * t.x + a0 * t.y;
+        x1[h + 1] = a1 * t.z - b1 * t.w;  x2[h + 1] = b1 * t.z + a1 * t.w;
+      }
+      u0 = pack8(x1);
+      u1 = pack8(x2);
+    }
+    const int slot = row % ring_rows;
+    const int s = swz(slot);
+    ring[slot * kChunks + (p ^ s)] = u0;
+    ring[slot * kChunks + ((p + 4) ^ s)] = u1;
+  }
+}
+
+// Sink rows 0..S-1 into a plain (unswizzled) buffer.
+template <bool ROT>
+__device__ __forceinline__ void stage_sinks(uint4* buf, int S, const __nv_bfloat16* src,
+                                            const float2* rope) {
+  for (int task = threadIdx.x; task < S * 4; task += blockDim.x) {
+    const int row = task >> 2, p = task & 3;
+    const uint4* g = reinterpret_cast<const uint4*>(src + (size_t)row * kD);
+    uint4 u0 = __ldg(g + p), u1 = __ldg(g + p + 4);
+    if (ROT) {
+      float x1[8], x2[8];
+      unpack8(u0, x1);
+      unpack8(u1, x2);
+      const float4* cs = reinterpret_cast<const float4*>(rope + (size_t)row * 32 + 8 * p);
+#pragma unroll
+      for (int h = 0; h < 8; h += 2) {
+        const float4 t = __ldg(cs + h / 2);
+        float a0 = x1[h], b0 = x2[h], a1 = x1[h + 1], b1 = x2[h + 1];
+        x1[h] = a0 * t.x - b0 * t.y;  x2[h] = b0 * t.x + a0 * t.y;
+        x1[h + 1] = a1 * t.z - b1 * t.w;  x2[h + 1] = b1 * t.z + a1 * t.w;
+      }
+      u0 = pack8(x1);
+      u1 = pack8(x2);
+    }
+    buf[row * kChunks + p] = u0;
+    buf[row * kChunks + p + 4] = u1;
+  }
+}
+
+__device__ __forceinline__ void sink_load(const uint4* buf, int s, int c, float (&x)[16]) {
+  unpack8(buf[s * kChunks + c], x);
+  unpack8(buf[s * kChunks + c + 4], x + 8);
+}
+
+}  // namespace fast
+}  // namespace sa

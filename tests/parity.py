@@ -4,8 +4,10 @@ the same seeded inputs and compare with the stated tolerances.
 Tolerances (written here, used by every parity test):
   fp32 inputs : max |GPU - oracle| <= 1e-5 on O, LSE, dQ, dK, dV;
                 |d alpha| relative error <= 1e-5 (it is a sum of many terms).
-  bf16 inputs : max |GPU - oracle| <= 1e-2 on O (stored as bf16) and on LSE
-                (fp32); relative Frobenius norm <= 5e-2 on dQ, dK, dV and
+  bf16 inputs : |GPU - oracle| <= 1e-2 + ulp_bf16(oracle)/2 elementwise on O
+                -- the 1e-2 bound applies to the computation, and O is stored
+                in bf16, whose rounding alone reaches 0.0078 for |O| in [2, 4)
+                and 0.0156 in [4, 8); max |GPU - oracle| <= 1e-2 on LSE (fp32); relative Frobenius norm <= 5e-2 on dQ, dK, dV and
                 relative error <= 5e-2 on d alpha.  The LSE bound follows from
                 the staged kernels keeping rotated K rows in bf16: a relative
                 rounding of 2^-9 per element gives score errors of about
@@ -41,14 +43,23 @@ def run_gpu_fwd(q, k, v, alpha, **kw):
     return o, lse
 
 
+def half_ulp_bf16(x):
+    """Half a bf16 unit in the last place of |x| (8 significant bits)."""
+    ax = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    return np.where(ax > 0, np.exp2(e - 8), 0.0)
+
+
 def check_fwd(o_gpu, lse_gpu, o_ref, lse_ref, dtype, what=""):
     tol = TOL[dtype]
     o_gpu, lse_gpu = to_np(o_gpu), to_np(lse_gpu)
     assert np.array_equal(np.isnan(o_gpu), np.isnan(o_ref)), f"{what}: NaN pattern of O"
     fin = ~np.isnan(o_ref)
-    err_o = np.abs(o_gpu - o_ref)[fin].max(initial=0.0)
+    store = half_ulp_bf16(o_ref) if dtype == torch.bfloat16 else 0.0
+    excess = (np.abs(o_gpu - o_ref) - store)[fin]
+    err_o = excess.max(initial=0.0)
     err_l = np.abs(lse_gpu - lse_ref)[~np.isnan(lse_ref)].max(initial=0.0)
-    assert err_o <= tol["o_abs"], f"{what}: O max abs err {err_o:.3e}"
+    assert err_o <= tol["o_abs"], f"{what}: O max abs err beyond bf16 storage {err_o:.3e}"
     assert err_l <= tol["lse_abs"], f"{what}: LSE max abs err {err_l:.3e}"
     return err_o, err_l
 
