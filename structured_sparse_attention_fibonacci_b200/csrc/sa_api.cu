@@ -4,6 +4,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <vector>
 
@@ -174,7 +175,10 @@ size_t sparse_attn_workspace_size(const sa_params* p, int backward) {
   sa::Problem pb;
   if (build_problem(p, &pb) != SA_OK) return 0;
   if (!backward) return 0;
-  return sa::general_bwd_layout(pb).total;
+  // enough for whichever backward path a call takes (see sparse_attn_force_general)
+  size_t need = sa::general_bwd_layout(pb).total;
+  if (sa::fast_bwd_supported(pb)) need = std::max(need, sa::fast_bwd_workspace(pb));
+  return need;
 }
 
 sa_status sparse_attn_fwd(const sa_params* p, const void* q, const void* k, const void* v,
@@ -223,7 +227,10 @@ sa_status sparse_attn_bwd(const sa_params* p, const void* q, const void* k, cons
   if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
   sa::BwdPtrs a = {q, k, v, o, dout, lse, alpha, dq, dk, dv, dalpha, rope, workspace};
   int launches = 0;
-  if (sa::launch_bwd_general(pb, a, st, &launches) != cudaSuccess) return SA_ERR_CUDA;
+  cudaError_t e = (!g_force_general && sa::fast_bwd_supported(pb))
+                      ? sa::launch_bwd_fast(pb, a, st, &launches)
+                      : sa::launch_bwd_general(pb, a, st, &launches);
+  if (e != cudaSuccess) return SA_ERR_CUDA;
   g_last_launches = launches;
   return SA_OK;
 }

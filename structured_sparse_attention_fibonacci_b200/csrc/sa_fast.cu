@@ -14,8 +14,8 @@
 //    then the offsets sorted by f).  Each member needs a contiguous row range;
 //    only rows below everything staged so far are fetched, into a ring of
 //    shared-memory rows, so every row of the tile's union is read from L2 once
-//    per pass.  K rows are rotated (RoPE) on the way in; rows are stored as
-//    bf16 with a 16-byte-chunk XOR swizzle.
+//    per pass.  K rows are rotated (RoPE) on the way in and kept as scaled
+//    fp16, V rows as bf16, with a 16-byte-chunk XOR swizzle.
 //  * An offset whose rows lie inside the window ("near") costs nothing: its
 //    score is the interpolation of two window scores, and its probability is
 //    folded into the two window weights used for PV.
@@ -55,7 +55,7 @@ __device__ __forceinline__ void window_scores(const uint4* ring, int ring_rows, 
   for (int u = 0; u < LC + 3; ++u) {
     const int row = max(ig + 3 - d0 - u, 0);
     float x[16];
-    ring_load(ring, row % ring_rows, c, x);
+    ring_load<true>(ring, row % ring_rows, c, x);
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int l = a + u - 3;
@@ -138,7 +138,9 @@ __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
   for (int e = t; e < (a.ring_rows + S) * kChunks; e += M) ring[e] = make_uint4(0, 0, 0, 0);
   const int S_rows = min(S, T);
 
-  // this lane's slice of its 4 queries, rotated and scaled
+  // this lane's slice of its 4 queries, rotated and scaled (times the inverse
+  // of the key staging factor)
+  const float qs = a.scale * kKeyUnstage;
   float q[4][16];
 #pragma unroll
   for (int qq = 0; qq < 4; ++qq) {
@@ -151,10 +153,10 @@ __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
 #pragma unroll
     for (int h = 0; h < 8; h += 2) {
       const float4 tt = __ldg(cs + h / 2);
-      q[qq][h] = (x1[h] * tt.x - x2[h] * tt.y) * a.scale;
-      q[qq][h + 8] = (x2[h] * tt.x + x1[h] * tt.y) * a.scale;
-      q[qq][h + 1] = (x1[h + 1] * tt.z - x2[h + 1] * tt.w) * a.scale;
-      q[qq][h + 9] = (x2[h + 1] * tt.z + x1[h + 1] * tt.w) * a.scale;
+      q[qq][h] = (x1[h] * tt.x - x2[h] * tt.y) * qs;
+      q[qq][h + 8] = (x2[h] * tt.x + x1[h] * tt.y) * qs;
+      q[qq][h + 1] = (x1[h + 1] * tt.z - x2[h + 1] * tt.w) * qs;
+      q[qq][h + 9] = (x2[h + 1] * tt.z + x1[h + 1] * tt.w) * qs;
     }
   }
 
@@ -180,7 +182,7 @@ __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       float x[16];
-      sink_load(sinkb, min(s0 + j, S - 1), c, x);
+      sink_load<true>(sinkb, min(s0 + j, S - 1), c, x);
 #pragma unroll
       for (int qq = 0; qq < 4; ++qq) acc[qq][j] = dot16(q[qq], x);
     }
@@ -208,7 +210,7 @@ __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
       if (u == 0 && !two) continue;
       const int row = max(ig - g.lo - 1 + u, 0);
       float x[16];
-      ring_load(ring, row % RB, c, x);
+      ring_load<true>(ring, row % RB, c, x);
       if (u <= 3) pb[u] = dot16(q[u], x);
       if (u >= 1) pa[u - 1] = dot16(q[u - 1], x);
     }

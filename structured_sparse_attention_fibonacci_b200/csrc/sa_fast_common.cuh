@@ -5,6 +5,7 @@
 
 #include "sa_device.cuh"
 #include "sa_internal.h"
+#include <cuda_fp16.h>
 
 namespace sa {
 namespace fast {
@@ -19,6 +20,33 @@ __device__ __forceinline__ void unpack8(const uint4 u, float* x) {
   x[4] = bf16lo(u.z); x[5] = bf16hi(u.z); x[6] = bf16lo(u.w); x[7] = bf16hi(u.w);
 }
 
+// Rotated K rows are staged as fp16 of (RoPE(K) * kKeyStage): fp16 keeps 8x
+// finer rounding than bf16 (2^-11 vs 2^-8 relative), and the 2^-8 factor
+// moves its range to |RoPE(K)| < 65504 * 256 (about 1.7e7).  Queries carry
+// the inverse factor, so scores come out unscaled.
+constexpr float kKeyStage = 1.f / 256.f;
+constexpr float kKeyUnstage = 256.f;
+
+__device__ __forceinline__ void unpack8_h(const uint4 u, float* x) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[e]));
+    x[2 * e] = f.x;
+    x[2 * e + 1] = f.y;
+  }
+}
+
+__device__ __forceinline__ uint4 pack8_h(const float* x) {
+  uint32_t w[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __half2 h = __floats2half2_rn(x[2 * e], x[2 * e + 1]);
+    w[e] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 __device__ __forceinline__ uint4 pack8(const float* x) {
   return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
                     pack_bf16x2(x[6], x[7]));
@@ -26,11 +54,17 @@ __device__ __forceinline__ uint4 pack8(const float* x) {
 
 __device__ __forceinline__ int swz(int slot) { return (slot >> 2) & 7; }
 
-// This lane's 16 dims of ring slot `slot`.
+// This lane's 16 dims of ring slot `slot` (F16: a staged rotated-K row).
+template <bool F16 = false>
 __device__ __forceinline__ void ring_load(const uint4* ring, int slot, int c, float (&x)[16]) {
   const int s = swz(slot);
-  unpack8(ring[slot * kChunks + (c ^ s)], x);
-  unpack8(ring[slot * kChunks + ((c + 4) ^ s)], x + 8);
+  if (F16) {
+    unpack8_h(ring[slot * kChunks + (c ^ s)], x);
+    unpack8_h(ring[slot * kChunks + ((c + 4) ^ s)], x + 8);
+  } else {
+    unpack8(ring[slot * kChunks + (c ^ s)], x);
+    unpack8(ring[slot * kChunks + ((c + 4) ^ s)], x + 8);
+  }
 }
 
 __device__ __forceinline__ float dot16(const float (&q)[16], const float (&x)[16]) {
@@ -90,11 +124,12 @@ __device__ __forceinline__ void stage_rows(uint4* ring, int ring_rows, const __n
       for (int h = 0; h < 8; h += 2) {
         const float4 t = __ldg(cs + h / 2);
         float a0 = x1[h], b0 = x2[h], a1 = x1[h + 1], b1 = x2[h + 1];
-        x1[h] = a0 * t.x - b0 * t.y;  x2[h] = b0 * t.x + a0 * t.y;
-        x1[h + 1] = a1 * t.z - b1 * t.w;  x2[h + 1] = b1 * t.z + a1 * t.w;
+        x1[h] = (a0 * t.x - b0 * t.y) * kKeyStage;  x2[h] = (b0 * t.x + a0 * t.y) * kKeyStage;
+        x1[h + 1] = (a1 * t.z - b1 * t.w) * kKeyStage;
+        x2[h + 1] = (b1 * t.z + a1 * t.w) * kKeyStage;
       }
-      u0 = pack8(x1);
-      u1 = pack8(x2);
+      u0 = pack8_h(x1);
+      u1 = pack8_h(x2);
     }
     const int slot = row % ring_rows;
     const int s = swz(slot);
@@ -120,20 +155,27 @@ __device__ __forceinline__ void stage_sinks(uint4* buf, int S, const __nv_bfloat
       for (int h = 0; h < 8; h += 2) {
         const float4 t = __ldg(cs + h / 2);
         float a0 = x1[h], b0 = x2[h], a1 = x1[h + 1], b1 = x2[h + 1];
-        x1[h] = a0 * t.x - b0 * t.y;  x2[h] = b0 * t.x + a0 * t.y;
-        x1[h + 1] = a1 * t.z - b1 * t.w;  x2[h + 1] = b1 * t.z + a1 * t.w;
+        x1[h] = (a0 * t.x - b0 * t.y) * kKeyStage;  x2[h] = (b0 * t.x + a0 * t.y) * kKeyStage;
+        x1[h + 1] = (a1 * t.z - b1 * t.w) * kKeyStage;
+        x2[h + 1] = (b1 * t.z + a1 * t.w) * kKeyStage;
       }
-      u0 = pack8(x1);
-      u1 = pack8(x2);
+      u0 = pack8_h(x1);
+      u1 = pack8_h(x2);
     }
     buf[row * kChunks + p] = u0;
     buf[row * kChunks + p + 4] = u1;
   }
 }
 
+template <bool F16 = false>
 __device__ __forceinline__ void sink_load(const uint4* buf, int s, int c, float (&x)[16]) {
-  unpack8(buf[s * kChunks + c], x);
-  unpack8(buf[s * kChunks + c + 4], x + 8);
+  if (F16) {
+    unpack8_h(buf[s * kChunks + c], x);
+    unpack8_h(buf[s * kChunks + c + 4], x + 8);
+  } else {
+    unpack8(buf[s * kChunks + c], x);
+    unpack8(buf[s * kChunks + c + 4], x + 8);
+  }
 }
 
 }  // namespace fast

@@ -484,6 +484,14 @@ BwdLayout general_bwd_layout(const Problem& pb) {
   return lay;
 }
 
+cudaError_t launch_reduce_dalpha(const float* part, int L, int per_layer, float* dalpha,
+                                 cudaStream_t st) {
+  trace_mark("reduce_dalpha", st, true);
+  k_reduce_dalpha<<<L, 256, 0, st>>>(part, per_layer, dalpha);
+  trace_mark("reduce_dalpha", st, false);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_rope_table(float2* tab, int T, int D, double base, cudaStream_t st) {
   const size_t n = (size_t)T * (D / 2);
   const int grid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
@@ -531,11 +539,11 @@ static cudaError_t bwd_t(const Problem& pb, const BwdPtrs& p, cudaStream_t st, i
   k_bwd_kv_general<T, D><<<grid, kGenWarps * 32, 0, st>>>(a);
   trace_mark("bwd_kv_general", st, false);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  trace_mark("reduce_dalpha", st, true);
-  k_reduce_dalpha<<<pb.L, 256, 0, st>>>(a.dal_part, pb.B * pb.H * a.n_tiles, p.dalpha);
-  trace_mark("reduce_dalpha", st, false);
+  if ((e = launch_reduce_dalpha(a.dal_part, pb.L, pb.B * pb.H * a.n_tiles, p.dalpha, st)) !=
+      cudaSuccess)
+    return e;
   *launches += 3;
-  return cudaGetLastError();
+  return cudaSuccess;
 }
 
 template <typename T>

@@ -52,6 +52,15 @@ bool fast_fwd_supported(const Problem& pb);
 size_t fast_fwd_smem(const Problem& pb, int* ring_rows, int* sc_stride);
 cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& a, cudaStream_t st, int* launches);
 
+// Staged bf16 / D=64 backward (sa_fast_bwd.cu).
+bool fast_bwd_supported(const Problem& pb);
+size_t fast_bwd_workspace(const Problem& pb);
+cudaError_t launch_bwd_fast(const Problem& pb, const BwdPtrs& a, cudaStream_t st, int* launches);
+
+// dalpha[l] = fixed-order sum of part[l * per_layer .. (l+1) * per_layer).
+cudaError_t launch_reduce_dalpha(const float* part, int L, int per_layer, float* dalpha,
+                                 cudaStream_t st);
+
 cudaError_t launch_rope_table(float2* tab, int T, int D, double base, cudaStream_t st);
 cudaError_t launch_fwd_general(const Problem& pb, const FwdPtrs& a, cudaStream_t st, int* launches);
 cudaError_t launch_bwd_general(const Problem& pb, const BwdPtrs& a, cudaStream_t st, int* launches);

@@ -177,3 +177,37 @@ def test_fast_path_is_the_one_dispatched():
     finally:
         sa.trace_enable(False)
     assert names == {"fwd_fast"}, names
+
+
+@pytest.mark.parametrize("case", FAST, ids=[c[0] for c in FAST])
+def test_fast_and_general_backward(case):
+    name, shape, W, S, alphas, offs = case
+    q, k, v, do = _inputs(shape, torch.bfloat16, seed=zlib.crc32(name.encode()) % 10000 + 1)
+    alpha = torch.tensor(alphas, dtype=torch.float32, device=DEV)
+    kw = dict(window=W, sinks=S, offsets=offs)
+    ref = oracle_bwd(q, k, v, do, alpha, **kw)
+    o, lse = run_gpu_fwd(q, k, v, alpha, **kw)
+    g_fast = [t.clone() for t in sa.bwd(q, k, v, o, lse, do, alpha, **kw)]
+    torch.cuda.synchronize()
+    check_bwd(g_fast, ref, torch.bfloat16, name + " (staged)")
+    sa.force_general(True)
+    try:
+        o, lse = run_gpu_fwd(q, k, v, alpha, **kw)
+        g_gen = sa.bwd(q, k, v, o, lse, do, alpha, **kw)
+        torch.cuda.synchronize()
+    finally:
+        sa.force_general(False)
+    check_bwd(g_gen, ref, torch.bfloat16, name + " (general)")
+
+
+def test_fast_backward_is_the_one_dispatched():
+    q, k, v, do = _inputs((1, 1, 1, 300, 64), torch.bfloat16, seed=6)
+    alpha = torch.tensor([1.0], device=DEV)
+    o, lse = run_gpu_fwd(q, k, v, alpha, window=12)
+    sa.trace_enable(True)
+    try:
+        sa.bwd(q, k, v, o, lse, do, alpha, window=12)
+        names = set(sa.trace_read())
+    finally:
+        sa.trace_enable(False)
+    assert names == {"bwd_q_fast", "bwd_kv_fast", "reduce_dalpha"}, names
