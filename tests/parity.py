@@ -3,12 +3,12 @@ the same seeded inputs and compare with the stated tolerances.
 
 Tolerances (written here, used by every parity test):
   fp32 inputs : max |GPU - oracle| <= 1e-5 on O, LSE, dQ, dK, dV;
-                |d alpha| relative error <= 1e-5 (it is a sum of many terms).
+                relative norm <= 1e-5 on the per-layer d-alpha vector.
   bf16 inputs : |GPU - oracle| <= 1e-2 + ulp_bf16(oracle)/2 elementwise on O
                 -- the 1e-2 bound applies to the computation, and O is stored
                 in bf16, whose rounding alone reaches 0.0078 for |O| in [2, 4)
                 and 0.0156 in [4, 8); max |GPU - oracle| <= 1e-2 on LSE (fp32); relative Frobenius norm <= 5e-2 on dQ, dK, dV and
-                relative error <= 5e-2 on d alpha.  The LSE bound follows from
+                on the per-layer d-alpha vector.  The LSE bound follows from
                 the staged kernels keeping rotated K rows in bf16: a relative
                 rounding of 2^-9 per element gives score errors of about
                 2^-9/sqrt(3) * |q_hat o k| ~ 1e-3 for N(0,1) inputs, a few 1e-3
@@ -78,14 +78,25 @@ def check_bwd(gpu, ref, dtype, what=""):
             e = rel_norm(g[fin], r[fin])
             assert e <= tol["grad_rel"], f"{what}: {name} rel-norm err {e:.3e}"
         out[name] = e
-    dal_g, dal_r = to_np(gpu[3]), np.asarray(ref[3])
+    out["dalpha"] = check_dalpha(gpu[3], ref[3], dtype, what)
+    return out
+
+
+def check_dalpha(dal_gpu, dal_ref, dtype, what=""):
+    """Relative norm of the per-layer d-alpha vector.  Each layer's value is a
+    sum of per-(batch, head) terms that are large (about 1e4 for the learned-
+    alpha workload) and of both signs, so a single layer's total can cancel to
+    a value far below its terms (layer 0 of that workload: -72.7, next to
+    1e5-scale layers); the norm over layers is the well-conditioned measure."""
+    tol = TOL[dtype]
+    dal_g, dal_r = to_np(dal_gpu), np.asarray(dal_ref, np.float64)
     fin = ~np.isnan(dal_r)
     assert np.array_equal(np.isnan(dal_g), ~fin), f"{what}: NaN pattern of dalpha"
-    e = np.abs(dal_g - dal_r)[fin] / np.maximum(np.abs(dal_r[fin]), 1e-3)
-    e = float(e.max(initial=0.0))
-    assert e <= tol["dal_rel"], f"{what}: dalpha rel err {e:.3e} ({dal_g} vs {dal_r})"
-    out["dalpha"] = e
-    return out
+    if not fin.any():
+        return 0.0
+    e = float(np.linalg.norm(dal_g[fin] - dal_r[fin]) / max(np.linalg.norm(dal_r[fin]), 1e-3))
+    assert e <= tol["dal_rel"], f"{what}: dalpha rel-norm err {e:.3e} ({dal_g} vs {dal_r})"
+    return e
 
 
 def oracle_fwd(q, k, v, alpha, **kw):
