@@ -128,6 +128,32 @@ sa_status sparse_attn_bwd(const sa_params* p, const void* q, const void* k, cons
                           const float* alpha, void* dq, void* dk, void* dv, float* dalpha,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Forward that allocates no device memory.  The paper has no counterpart: this
+ * entry point exists for callers that cannot let a library call cudaMalloc --
+ * applications whose device memory belongs to a pooling allocator that must
+ * account for every byte, and embedders or latency-critical services that
+ * forbid allocation after start-up.  It computes exactly what sparse_attn_fwd
+ * computes (same arguments minus the workspace), but keeps its only scratch,
+ * the RoPE cos/sin table, in a fixed file-scope device array of
+ * SA_NOALLOC_SCRATCH_BYTES (8 MiB) that every GPU loading this library holds
+ * until the process exits.
+ *   Limit: T * (D/2) * 8 bytes must fit in SA_NOALLOC_SCRATCH_BYTES (for D=64,
+ *   T <= 32768); larger problems return SA_ERR_UNSUPPORTED before any work.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   Sharing: every call on a device uses the same array and rewrites the part
+ *   it needs on `stream` before reading it; calls that overlap on the GPU
+ *   (for example on two streams) race on the array and must be serialised by
+ *   the caller.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define SA_NOALLOC_SCRATCH_BYTES (8u << 20)
+sa_status sparse_attn_fwd_noalloc(const sa_params* p, const void* q, const void* k,
+                                  const void* v, const float* alpha, void* o, float* lse,
+                                  void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* sparse_attn_status_string(sa_status s);
 

@@ -31,7 +31,8 @@ MAX_SINKS = 16
 
 EXPORTED = ("sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_workspace_size",
             "sparse_attn_status_string", "sparse_attn_last_launch_count",
-            "sparse_attn_trace_enable", "sparse_attn_trace_read", "sparse_attn_force_general")
+            "sparse_attn_trace_enable", "sparse_attn_trace_read", "sparse_attn_force_general",
+            "sparse_attn_fwd_noalloc")
 
 
 class SaParams(ctypes.Structure):
@@ -69,6 +70,8 @@ def lib():
         L.sparse_attn_bwd.restype = ctypes.c_int
         L.sparse_attn_bwd.argtypes = [P, vp, vp, vp, vp, fp, vp, fp, vp, vp, vp, fp, vp,
                                       ctypes.c_size_t, vp]
+        L.sparse_attn_fwd_noalloc.restype = ctypes.c_int
+        L.sparse_attn_fwd_noalloc.argtypes = [P, vp, vp, vp, fp, vp, fp, vp]
         L.sparse_attn_status_string.restype = ctypes.c_char_p
         L.sparse_attn_status_string.argtypes = [ctypes.c_int]
         L.sparse_attn_last_launch_count.restype = ctypes.c_int32
@@ -182,6 +185,30 @@ def fwd(q, k, v, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0, sc
     st = L.sparse_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(out),
                            _ptr(lse), _ptr(ws), ws_n, _stream_handle(stream))
     _check("sparse_attn_fwd", st)
+    return out, lse
+
+
+def fwd_noalloc(q, k, v, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0,
+                scale=0.0, out=None, lse=None, want_lse=True, stream=None):
+    """Forward through sparse_attn_fwd_noalloc: the library allocates nothing.
+
+    For callers that cannot let a library allocate device memory (a pooling
+    allocator that must see every byte, or no allocation after start-up).  The
+    RoPE table lives in a fixed 8 MiB device array (T * D/2 * 8 bytes must fit);
+    calls that overlap on the GPU share that array and must be serialised.
+    Output buffers may be passed in; otherwise they are allocated here by torch,
+    on the caller's side of the boundary.
+    """
+    shape, dtype, dev = tuple(q.shape), q.dtype, q.device
+    if lse is None and want_lse:
+        lse = torch.empty(shape[:4], dtype=torch.float32, device=dev)
+    out = torch.empty_like(q) if out is None else out
+    _check_tensors(shape, dtype, dev, q=q, k=k, v=v, o=out, alpha=alpha, lse=lse)
+    p = make_params(shape, dtype, window=window, offsets=offsets, sinks=sinks,
+                    rope_base=rope_base, scale=scale)
+    st = lib().sparse_attn_fwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                       _ptr(out), _ptr(lse), _stream_handle(stream))
+    _check("sparse_attn_fwd_noalloc", st)
     return out, lse
 
 

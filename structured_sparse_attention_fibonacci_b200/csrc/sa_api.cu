@@ -103,6 +103,14 @@ cudaEvent_t take_event() {
 }  // namespace
 
 namespace sa {
+sa_status validate_params(const sa_params* p, Problem* pb) { return build_problem(p, pb); }
+
+cudaError_t launch_fwd_dispatch(const Problem& pb, const FwdPtrs& a, cudaStream_t st,
+                                int* launches) {
+  return (!g_force_general && fast_fwd_supported(pb)) ? launch_fwd_fast(pb, a, st, launches)
+                                                      : launch_fwd_general(pb, a, st, launches);
+}
+
 void trace_mark(const char* kernel, cudaStream_t st, bool begin) {
   std::lock_guard<std::mutex> lock(g_trace_mu);
   if (!g_trace_on) return;

@@ -41,6 +41,13 @@ struct BwdLayout {
 
 BwdLayout general_bwd_layout(const Problem& pb);
 
+// Argument validation shared by every C entry point (defined in sa_api.cu).
+sa_status validate_params(const sa_params* p, Problem* pb);
+// Forward dispatch shared by the C entry points: the staged kernel where it
+// applies (and the general kernels are not forced), else the general kernel.
+cudaError_t launch_fwd_dispatch(const Problem& pb, const FwdPtrs& a, cudaStream_t st,
+                                int* launches);
+
 // Tracing hook: brackets one kernel launch with events when tracing is on.
 // Call with begin = true just before the launch and false just after it.
 void trace_mark(const char* kernel, cudaStream_t st, bool begin);

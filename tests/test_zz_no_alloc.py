@@ -1,0 +1,71 @@
+"""sparse_attn_fwd_noalloc, the forward for callers that cannot let a library
+allocate device memory (a pooling allocator that must see every byte, or no
+allocation after start-up), checked through the C ABI against the regular
+sparse_attn_fwd on the same inputs.
+
+The outputs are allocated here by the test, before the call; the entry point
+itself allocates nothing and keeps its RoPE table in a fixed device array.
+Consecutive calls use different shapes, so each one has to rewrite the part of
+that shared array it reads.
+"""
+import ctypes
+
+import pytest
+import torch
+
+import structured_sparse_attention_fibonacci_b200 as sa
+
+DEV = "cuda"
+
+# (dtype, (L, B, H, T, D), window, sinks, alphas); O / LSE tolerance as in the
+# parity tests: fp32 1e-5, bf16 1e-2 (both calls run the same kernels here)
+CASES = [
+    (torch.bfloat16, (2, 1, 2, 300, 64), 12, 2, [0.5666667, 1.5]),
+    (torch.float32, (1, 1, 2, 64, 16), 6, 0, [1.0]),
+    (torch.bfloat16, (1, 2, 1, 1100, 64), 12, 0, [1.1234]),
+]
+TOL = {torch.float32: 1e-5, torch.bfloat16: 1e-2}
+
+
+def _inputs(shape, dtype, seed):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    return [torch.randn(shape, generator=g).to(dtype).to(DEV) for _ in range(3)]
+
+
+def _call_noalloc(q, k, v, alpha, o, lse, **kw):
+    p = sa.make_params(tuple(q.shape), q.dtype, **kw)
+    st = sa.lib().sparse_attn_fwd_noalloc(
+        ctypes.byref(p), ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+        ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(alpha.data_ptr()),
+        ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(lse.data_ptr()),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == sa.SA_OK, sa.status_string(st)
+
+
+def _check_case(i, case):
+    dtype, shape, W, S, alphas = case
+    q, k, v = _inputs(shape, dtype, seed=100 + i)
+    alpha = torch.tensor(alphas, dtype=torch.float32, device=DEV)
+    kw = dict(window=W, sinks=S)
+    o_ref, lse_ref = sa.fwd(q, k, v, alpha, **kw)
+    o = torch.empty_like(q)
+    lse = torch.empty(shape[:4], dtype=torch.float32, device=DEV)
+    _call_noalloc(q, k, v, alpha, o, lse, **kw)
+    torch.cuda.synchronize()
+    assert (o.float() - o_ref.float()).abs().max().item() <= TOL[dtype]
+    assert (lse - lse_ref).abs().max().item() <= TOL[dtype]
+
+
+@pytest.mark.gpu
+def test_noalloc_forward_matches_the_regular_forward_on_calls_in_a_row():
+    for i, case in enumerate(CASES):
+        _check_case(i, case)
+    _check_case(0, CASES[0])          # first shape again, after the others
+
+
+def test_noalloc_rejects_tables_beyond_its_array_before_any_work():
+    p = sa.make_params((1, 1, 1, 40000, 64), torch.bfloat16, window=12)
+    dummy = ctypes.c_void_p(1 << 20)   # never dereferenced: the size check comes first
+    st = sa.lib().sparse_attn_fwd_noalloc(ctypes.byref(p), dummy, dummy, dummy, dummy, dummy,
+                                          dummy, None)
+    assert st == sa.SA_ERR_UNSUPPORTED
