@@ -55,7 +55,7 @@ __device__ __forceinline__ void window_scores(const uint4* ring, int ring_rows, 
   for (int u = 0; u < LC + 3; ++u) {
     const int row = max(ig + 3 - d0 - u, 0);
     float x[16];
-    ring_load<true>(ring, row % ring_rows, c, x);
+    ring_load<true>(ring, row & (ring_rows - 1), c, x);
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int l = a + u - 3;
@@ -81,7 +81,7 @@ __device__ __forceinline__ void window_pv(const uint4* ring, int ring_rows, int 
   for (int u = 0; u < LC + 3; ++u) {
     const int row = max(ig + 3 - d0 - u, 0);
     float x[16];
-    ring_load(ring, row % ring_rows, c, x);
+    ring_load(ring, row & (ring_rows - 1), c, x);
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int l = a + u - 3;
@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
       if (u == 0 && !two) continue;
       const int row = max(ig - g.lo - 1 + u, 0);
       float x[16];
-      ring_load<true>(ring, row % RB, c, x);
+      ring_load<true>(ring, row & (RB - 1), c, x);
       if (u <= 3) pb[u] = dot16(q[u], x);
       if (u >= 1) pa[u - 1] = dot16(q[u - 1], x);
     }
@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
       if (u == 0 && !two) continue;
       const int row = max(ig - g.lo - 1 + u, 0);
       float x[16];
-      ring_load(ring, row % RB, c, x);
+      ring_load(ring, row & (RB - 1), c, x);
       if (u <= 3 && two) axpy16(o[u], p[u] * g.w, x);
       if (u >= 1) axpy16(o[u - 1], p[u - 1] * g.wa, x);
     }
@@ -334,7 +334,8 @@ bool fast_fwd_supported(const Problem& pb) {
 }
 
 size_t fast_fwd_smem(const Problem& pb, int* ring_rows, int* sc_stride) {
-  const int rr = ((std::max(kFastM + pb.W - 1, kFastM + 2) + 31) / 32) * 32;
+  int rr = 32;   // a power of two: ring slots are row & (rr - 1)
+  while (rr < std::max(kFastM + pb.W - 1, kFastM + 2)) rr *= 2;
   // odd stride: the 8 lane groups of a warp read rows 4 apart, and the 32
   // owner lanes read 32 consecutive rows, without shared-memory bank conflicts
   const int n_slot = pb.W + pb.S + pb.n_off;

@@ -104,7 +104,7 @@ __device__ __forceinline__ void window_dots(const uint4* ring, int RB, int ig, i
   for (int u = 0; u < LC + 3; ++u) {
     const int row = max(ig + 3 - d0 - u, 0);
     float x[16];
-    ring_load<F16>(ring, row % RB, c, x);
+    ring_load<F16>(ring, row & (RB - 1), c, x);
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int l = a + u - 3;
@@ -130,7 +130,7 @@ __device__ __forceinline__ void window_axpy(const uint4* ring, int RB, int ig, i
   for (int u = 0; u < LC + 3; ++u) {
     const int row = max(ig + 3 - d0 - u, 0);
     float x[16];
-    ring_load<F16>(ring, row % RB, c, x);
+    ring_load<F16>(ring, row & (RB - 1), c, x);
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int l = a + u - 3;
@@ -198,7 +198,7 @@ __device__ __forceinline__ void member_dots(const FastBwdArgs& a, uint4* ring, u
     for (int u = 0; u < 5; ++u) {
       const int row = max(ig - g.lo - 1 + u, 0);
       float y[16];
-      ring_load<ROT>(ring, row % RB, c, y);
+      ring_load<ROT>(ring, row & (RB - 1), c, y);
       if (u <= 3) pb[u] = dot16(x[u], y);
       if (u >= 1) pa[u - 1] = dot16(x[u - 1], y);
     }
@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
         if (u == 0 && !two) continue;
         const int row = max(ig - g.lo - 1 + u, 0);
         float y[16];
-        ring_load<true>(ring, row % RB, c, y);
+        ring_load<true>(ring, row & (RB - 1), c, y);
         if (u <= 3 && two) axpy16(x[u], gq[u] * g.w, y);
         if (u >= 1) axpy16(x[u - 1], gq[u - 1] * g.wa, y);
       }
@@ -503,15 +503,23 @@ __device__ __forceinline__ void stage_sources(const FastBwdArgs& a, uint4* ring,
         u1 = pack8(x2);
       }
     }
-    const int slot = row % RB, s = swz(slot);
+    const int slot = row & (RB - 1), s = swz(slot);
     ring[slot * kChunks + (p ^ s)] = u0;
     ring[slot * kChunks + ((p + 4) ^ s)] = u1;
   }
-  const int nw = (hi_row - lo_row) * NW;
-  for (int e = threadIdx.x; e < nw; e += blockDim.x) {
-    const int row = lo_row + e / NW, j = e % NW;
-    const float w = row < T ? __bfloat162float(wsrc[(size_t)row * a.slot_pitch + j]) : 0.f;
-    wring[(row % RB) * a.wpitch + j] = w;
+  // weights: 8 lanes per row, one 16-byte chunk (8 bf16) per lane and step
+  const int n_ch = (NW + 7) / 8;
+  for (int row = lo_row + (int)(threadIdx.x >> 3); row < hi_row; row += blockDim.x >> 3) {
+    float* dst = wring + (row & (RB - 1)) * a.wpitch;
+    for (int ch = threadIdx.x & 7; ch < n_ch; ch += 8) {
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (row < T) u = __ldg(reinterpret_cast<const uint4*>(wsrc + (size_t)row * a.slot_pitch) + ch);
+      float w8[8];
+      unpack8(u, w8);
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        if (ch * 8 + e < NW) dst[ch * 8 + e] = w8[e];
+    }
   }
 }
 
@@ -537,7 +545,7 @@ __device__ __forceinline__ void key_pass(const FastBwdArgs& a, uint4* ring, floa
 #define SA_KEY_WINDOW(LC)                                                        \
     {                                                                            \
       _Pragma("unroll") for (int u = 0; u < LC + 3; ++u) {                       \
-        const int slot = (rg + d0 + u) % RB;                                     \
+        const int slot = (rg + d0 + u) & (RB - 1);                                     \
         float y[16];                                                             \
         ring_load(ring, slot, c, y);                                             \
         _Pragma("unroll") for (int kk = 0; kk < 4; ++kk) {                       \
@@ -566,7 +574,7 @@ __device__ __forceinline__ void key_pass(const FastBwdArgs& a, uint4* ring, floa
     }
 #pragma unroll
     for (int u = 0; u < 5; ++u) {
-      const int slot = (rg + g.lo + u) % RB;
+      const int slot = (rg + g.lo + u) & (RB - 1);
       float y[16];
       ring_load(ring, slot, c, y);
       const float gk = wring[slot * wp + W + kk];
@@ -666,7 +674,8 @@ struct FastBwdLayout {
 FastBwdLayout fast_bwd_layout(const Problem& pb) {
   constexpr int M = kFastM;
   FastBwdLayout L;
-  L.ring_rows = ((std::max(M + pb.W - 1, M + 2) + 31) / 32) * 32;
+  L.ring_rows = 32;   // a power of two: ring slots are row & (ring_rows - 1)
+  while (L.ring_rows < std::max(M + pb.W - 1, M + 2)) L.ring_rows *= 2;
   const int n_slot = pb.W + pb.S + pb.n_off;
   L.sc_stride = n_slot | 1;
   const int NW = pb.W + pb.n_off;

@@ -67,19 +67,26 @@ __device__ __forceinline__ void ring_load(const uint4* ring, int slot, int c, fl
   }
 }
 
+// Dot product and axpy over a lane's 16 dims with packed fp32 FMAs
+// (two per instruction).
 __device__ __forceinline__ float dot16(const float (&q)[16], const float (&x)[16]) {
-  float a = 0.f, b = 0.f;
+  float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int h = 0; h < 16; h += 2) {
-    a = fmaf(q[h], x[h], a);
-    b = fmaf(q[h + 1], x[h + 1], b);
+  for (int h = 0; h < 16; h += 4) {
+    a = __ffma2_rn(make_float2(q[h], q[h + 1]), make_float2(x[h], x[h + 1]), a);
+    b = __ffma2_rn(make_float2(q[h + 2], q[h + 3]), make_float2(x[h + 2], x[h + 3]), b);
   }
-  return a + b;
+  return (a.x + b.x) + (a.y + b.y);
 }
 
 __device__ __forceinline__ void axpy16(float (&o)[16], float p, const float (&x)[16]) {
+  const float2 pp = make_float2(p, p);
 #pragma unroll
-  for (int h = 0; h < 16; ++h) o[h] = fmaf(p, x[h], o[h]);
+  for (int h = 0; h < 16; h += 2) {
+    const float2 r = __ffma2_rn(pp, make_float2(x[h], x[h + 1]), make_float2(o[h], o[h + 1]));
+    o[h] = r.x;
+    o[h + 1] = r.y;
+  }
 }
 
 // p[q][l] are partial sums held by the 4 lanes of a group (lane c = 2*hi+lo);
@@ -131,7 +138,7 @@ __device__ __forceinline__ void stage_rows(uint4* ring, int ring_rows, const __n
       u0 = pack8_h(x1);
       u1 = pack8_h(x2);
     }
-    const int slot = row % ring_rows;
+    const int slot = row & (ring_rows - 1);   // ring_rows is a power of two
     const int s = swz(slot);
     ring[slot * kChunks + (p ^ s)] = u0;
     ring[slot * kChunks + ((p + 4) ^ s)] = u1;
