@@ -45,7 +45,8 @@ struct FastArgs {
 // (row ig+q) takes row u at lag d0 + (q + u - 3).
 template <int LC>
 __device__ __forceinline__ void window_scores(const uint4* ring, int ring_rows, int ig, int d0,
-                                              int c, const float (&q)[4][16], float* sc_row) {
+                                              int c, const float (&q)[4][16], float* sc_row,
+                                              int i_own, float& mx) {
   float acc[4][LC];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
@@ -65,7 +66,10 @@ __device__ __forceinline__ void window_scores(const uint4* ring, int ring_rows, 
   float out[LC];
   reduce_scatter4<LC>(acc, out, c);
 #pragma unroll
-  for (int l = 0; l < LC; ++l) sc_row[d0 + l] = out[l];
+  for (int l = 0; l < LC; ++l) {
+    sc_row[d0 + l] = out[l];
+    if (i_own - (d0 + l) >= 0) mx = fmaxf(mx, out[l]);
+  }
 }
 
 // Window PV for lags [d0, d0 + LC) with weights sc[query][lag].
@@ -88,6 +92,20 @@ __device__ __forceinline__ void window_pv(const uint4* ring, int ring_rows, int 
       if (l >= 0 && l < LC) axpy16(o[a], pw[a][l], x);
     }
   }
+}
+
+// Rows a far offset's member needs for the tile [i0, i0 + M): [lo, hi).
+__device__ __forceinline__ int far_seg_lo(const OffGeo& g, int i0) {
+  return max(0, i0 - g.lo - (g.w != 0.f ? 1 : 0));
+}
+__device__ __forceinline__ int far_seg_hi(const OffGeo& g, int i0, int T) {
+  return max(0, min(T, i0 + kFastM - g.lo));
+}
+// Next offset after k that is not folded into the window (n_off when none).
+__device__ __forceinline__ int next_far(const int* s_fold, int k, int n_off) {
+  ++k;
+  while (k < n_off && s_fold[k]) ++k;
+  return k;
 }
 
 __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
@@ -161,6 +179,8 @@ __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
   }
 
   const int lr = 4 * gid + c;                  // this lane's query, tile-local
+  const int i_own = ig + c;                    // ... and its position
+  float mx = -INFINITY;                        // running max of its valid scores
   float* my_sc = sc + (size_t)lr * a.sc_stride;
   const int win_lo = max(0, i0 - W + 1), win_hi = min(T, i0 + M);
   const int RB = a.ring_rows;
@@ -172,10 +192,10 @@ __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
   __syncthreads();
   {
     int d0 = 0;
-    while (W - d0 >= 8) { window_scores<8>(ring, RB, ig, d0, c, q, my_sc); d0 += 8; }
-    if (W - d0 >= 4) { window_scores<4>(ring, RB, ig, d0, c, q, my_sc); d0 += 4; }
-    if (W - d0 >= 2) { window_scores<2>(ring, RB, ig, d0, c, q, my_sc); d0 += 2; }
-    if (W - d0 >= 1) { window_scores<1>(ring, RB, ig, d0, c, q, my_sc); d0 += 1; }
+    while (W - d0 >= 8) { window_scores<8>(ring, RB, ig, d0, c, q, my_sc, i_own, mx); d0 += 8; }
+    if (W - d0 >= 4) { window_scores<4>(ring, RB, ig, d0, c, q, my_sc, i_own, mx); d0 += 4; }
+    if (W - d0 >= 2) { window_scores<2>(ring, RB, ig, d0, c, q, my_sc, i_own, mx); d0 += 2; }
+    if (W - d0 >= 1) { window_scores<1>(ring, RB, ig, d0, c, q, my_sc, i_own, mx); d0 += 1; }
   }
   for (int s0 = 0; s0 < S; s0 += 4) {
     float acc[4][4];
@@ -190,77 +210,92 @@ __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
     reduce_scatter4<4>(acc, out, c);
 #pragma unroll
     for (int j = 0; j < 4; ++j)
-      if (s0 + j < S) my_sc[W + s0 + j] = out[j];
+      if (s0 + j < S) {
+        my_sc[W + s0 + j] = out[j];
+        if (s0 + j <= i_own) mx = fmaxf(mx, out[j]);
+      }
   }
-  int low = win_lo;
-  for (int kk = 0; kk < n_off; ++kk) {
-    if (s_fold[kk]) continue;                  // CTA-uniform
-    const OffGeo g = sg[kk];
-    const int two = g.w != 0.f;
-    const int seg_lo = max(0, i0 - g.lo - two), seg_hi = min(T, i0 + M - g.lo);
-    if (seg_lo < low && seg_lo < seg_hi) {
-      __syncthreads();
-      stage_rows<true>(ring, RB, K, a.rope, seg_lo, min(seg_hi, low));
-      low = seg_lo;
-      __syncthreads();
-    }
-    float pa[4] = {0.f, 0.f, 0.f, 0.f}, pb[4] = {0.f, 0.f, 0.f, 0.f};
+  // far offsets, staged in batches: consecutive members whose rows span at
+  // most RB rows share one staging round and are computed back to back
+  {
+    int low = win_lo;
+    int kk = next_far(s_fold, -1, n_off);
+    while (kk < n_off) {
+      const int hi = far_seg_hi(sg[kk], i0, T);
+      int last = kk, nx = next_far(s_fold, kk, n_off);
+      while (nx < n_off && hi - far_seg_lo(sg[nx], i0) <= RB) {
+        last = nx;
+        nx = next_far(s_fold, nx, n_off);
+      }
+      // rows the batch needs: [lo_row, hi); only those below `low` are new
+      const int lo_row = far_seg_lo(sg[last], i0);
+      if (lo_row < low && lo_row < hi) {
+        __syncthreads();
+        stage_rows<true>(ring, RB, K, a.rope, lo_row, min(hi, low));
+        low = lo_row;
+        __syncthreads();
+      }
+      for (int m = kk; m < nx; m = next_far(s_fold, m, n_off)) {
+        const OffGeo g = sg[m];
+        const int two = g.w != 0.f;
+        float pa[4] = {0.f, 0.f, 0.f, 0.f}, pb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int u = 0; u < 5; ++u) {
-      if (u == 0 && !two) continue;
-      const int row = max(ig - g.lo - 1 + u, 0);
-      float x[16];
-      ring_load<true>(ring, row & (RB - 1), c, x);
-      if (u <= 3) pb[u] = dot16(q[u], x);
-      if (u >= 1) pa[u - 1] = dot16(q[u - 1], x);
-    }
-    float part[4][1];
+        for (int u = 0; u < 5; ++u) {
+          if (u == 0 && !two) continue;
+          const int row = max(ig - g.lo - 1 + u, 0);
+          float x[16];
+          ring_load<true>(ring, row & (RB - 1), c, x);
+          if (u <= 3) pb[u] = dot16(q[u], x);
+          if (u >= 1) pa[u - 1] = dot16(q[u - 1], x);
+        }
+        float part[4][1];
 #pragma unroll
-    for (int qq = 0; qq < 4; ++qq) part[qq][0] = g.wa * pa[qq] + g.w * pb[qq];
-    float out[1];
-    reduce_scatter4<1>(part, out, c);
-    my_sc[W + S + kk] = out[0];
+        for (int qq = 0; qq < 4; ++qq) part[qq][0] = g.wa * pa[qq] + g.w * pb[qq];
+        float out[1];
+        reduce_scatter4<1>(part, out, c);
+        my_sc[W + S + m] = out[0];
+        if (i_own - g.c >= 0) mx = fmaxf(mx, out[0]);
+      }
+      kk = nx;
+    }
   }
   __syncthreads();
 
   // ---------------- softmax (owner lane of each query) ----------------
+  // The running max was taken as scores were produced; one pass turns scores
+  // into unnormalised weights e = exp(score - max); 1/sum is applied to O.
+  float inv_l = 0.f;
   {
-    const int i = ig + c;
+    const int i = i_own;
     if (i < T) {
-      for (int kk = 0; kk < n_off; ++kk) {
+      for (int kk = 0; kk < n_off; ++kk) {    // near offsets: from two window scores
         if (!s_fold[kk]) continue;
         const OffGeo g = sg[kk];
-        float s = g.wa * my_sc[g.lo];
-        if (g.w != 0.f) s += g.w * my_sc[g.lo + 1];
-        my_sc[W + S + kk] = s;
+        float sv = g.wa * my_sc[g.lo];
+        if (g.w != 0.f) sv += g.w * my_sc[g.lo + 1];
+        my_sc[W + S + kk] = sv;
+        if (i - g.c >= 0) mx = fmaxf(mx, sv);
       }
-      float m = -INFINITY;
-      for (int d = 0; d < W; ++d) if (i - d >= 0) m = fmaxf(m, my_sc[d]);
-      for (int s = 0; s < S; ++s) if (s <= i) m = fmaxf(m, my_sc[W + s]);
-      for (int kk = 0; kk < n_off; ++kk) if (i - sg[kk].c >= 0) m = fmaxf(m, my_sc[W + S + kk]);
       float l = 0.f;
       for (int d = 0; d < W; ++d) {
-        const float p = (i - d >= 0) ? __expf(my_sc[d] - m) : 0.f;
-        my_sc[d] = p; l += p;
+        const float e = (i - d >= 0) ? __expf(my_sc[d] - mx) : 0.f;
+        my_sc[d] = e; l += e;
       }
-      for (int s = 0; s < S; ++s) {
-        const float p = (s <= i) ? __expf(my_sc[W + s] - m) : 0.f;
-        my_sc[W + s] = p; l += p;
+      for (int sk = 0; sk < S; ++sk) {
+        const float e = (sk <= i) ? __expf(my_sc[W + sk] - mx) : 0.f;
+        my_sc[W + sk] = e; l += e;
       }
       for (int kk = 0; kk < n_off; ++kk) {
-        const float p = (i - sg[kk].c >= 0) ? __expf(my_sc[W + S + kk] - m) : 0.f;
-        my_sc[W + S + kk] = p; l += p;
-      }
-      const float inv = 1.f / l;
-      for (int d = 0; d < W + S + n_off; ++d) my_sc[d] *= inv;
-      for (int kk = 0; kk < n_off; ++kk) {     // fold near offsets into window weights
-        if (!s_fold[kk]) continue;
         const OffGeo g = sg[kk];
-        const float p = my_sc[W + S + kk];
-        my_sc[g.lo] += g.wa * p;
-        if (g.w != 0.f) my_sc[g.lo + 1] += g.w * p;
+        const float e = (i - g.c >= 0) ? __expf(my_sc[W + S + kk] - mx) : 0.f;
+        my_sc[W + S + kk] = e; l += e;
+        if (s_fold[kk]) {                      // fold into the two window weights
+          my_sc[g.lo] += g.wa * e;
+          if (g.w != 0.f) my_sc[g.lo + 1] += g.w * e;
+        }
       }
-      if (a.lse) a.lse[(size_t)unit * T + i] = m + __logf(l);
+      inv_l = 1.f / l;
+      if (a.lse) a.lse[(size_t)unit * T + i] = mx + __logf(l);
     } else {
       for (int d = 0; d < W + S + n_off; ++d) my_sc[d] = 0.f;
     }
@@ -290,31 +325,51 @@ __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
 #pragma unroll
     for (int qq = 0; qq < 4; ++qq) axpy16(o[qq], grp_sc[qq * a.sc_stride + W + s], x);
   }
-  low = win_lo;
-  for (int kk = 0; kk < n_off; ++kk) {
-    if (s_fold[kk]) continue;
-    const OffGeo g = sg[kk];
-    const int two = g.w != 0.f;
-    const int seg_lo = max(0, i0 - g.lo - two), seg_hi = min(T, i0 + M - g.lo);
-    if (seg_lo < low && seg_lo < seg_hi) {
-      __syncthreads();
-      stage_rows<false>(ring, RB, V, a.rope, seg_lo, min(seg_hi, low));
-      low = seg_lo;
-      __syncthreads();
-    }
-    float p[4];
+  {
+    int low = win_lo;
+    int kk = next_far(s_fold, -1, n_off);
+    while (kk < n_off) {
+      const int hi = far_seg_hi(sg[kk], i0, T);
+      int last = kk, nx = next_far(s_fold, kk, n_off);
+      while (nx < n_off && hi - far_seg_lo(sg[nx], i0) <= RB) {
+        last = nx;
+        nx = next_far(s_fold, nx, n_off);
+      }
+      const int lo_row = far_seg_lo(sg[last], i0);
+      if (lo_row < low && lo_row < hi) {
+        __syncthreads();
+        stage_rows<false>(ring, RB, V, a.rope, lo_row, min(hi, low));
+        low = lo_row;
+        __syncthreads();
+      }
+      for (int m = kk; m < nx; m = next_far(s_fold, m, n_off)) {
+        const OffGeo g = sg[m];
+        const int two = g.w != 0.f;
+        float p[4];
 #pragma unroll
-    for (int qq = 0; qq < 4; ++qq) p[qq] = grp_sc[qq * a.sc_stride + W + S + kk];
+        for (int qq = 0; qq < 4; ++qq) p[qq] = grp_sc[qq * a.sc_stride + W + S + m];
 #pragma unroll
-    for (int u = 0; u < 5; ++u) {
-      if (u == 0 && !two) continue;
-      const int row = max(ig - g.lo - 1 + u, 0);
-      float x[16];
-      ring_load(ring, row & (RB - 1), c, x);
-      if (u <= 3 && two) axpy16(o[u], p[u] * g.w, x);
-      if (u >= 1) axpy16(o[u - 1], p[u - 1] * g.wa, x);
+        for (int u = 0; u < 5; ++u) {
+          if (u == 0 && !two) continue;
+          const int row = max(ig - g.lo - 1 + u, 0);
+          float x[16];
+          ring_load(ring, row & (RB - 1), c, x);
+          if (u <= 3 && two) axpy16(o[u], p[u] * g.w, x);
+          if (u >= 1) axpy16(o[u - 1], p[u - 1] * g.wa, x);
+        }
+      }
+      kk = nx;
     }
   }
+
+  // 1 / sum of the weights, from each query's owner lane (lane 4*gid + qq)
+  float inv[4];
+#pragma unroll
+  for (int qq = 0; qq < 4; ++qq) inv[qq] = __shfl_sync(0xffffffffu, inv_l, (t & 28) + qq);
+#pragma unroll
+  for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+    for (int h = 0; h < 16; ++h) o[qq][h] *= inv[qq];
 
 #pragma unroll
   for (int qq = 0; qq < 4; ++qq) {

@@ -61,6 +61,19 @@ __device__ __forceinline__ int cta_geometry_bwd(const FastBwdArgs& a, int layer,
   return __syncthreads_or(bad);
 }
 
+// Next offset after k that the backward does not fold (n_off when none).
+__device__ __forceinline__ int next_far(const int* s_fold, int k, int n_off) {
+  ++k;
+  while (k < n_off && s_fold[k]) ++k;
+  return k;
+}
+// Rows a far member needs on the query side for the tile [i0, i0 + M), both
+// interpolation rows (the d-alpha term reads row i-lo-1 even when w == 0).
+__device__ __forceinline__ int qseg_lo(const OffGeo& g, int i0) { return max(0, i0 - g.lo - 1); }
+__device__ __forceinline__ int qseg_hi(const OffGeo& g, int i0, int T) {
+  return max(0, min(T, i0 + kFastM - g.lo));
+}
+
 // Load this lane's 16 dims of 4 consecutive rows of X (bf16 [T][64]), rows
 // clamped to T-1; optionally rotated (RoPE at the row's position) and scaled.
 template <bool ROT>
@@ -94,7 +107,8 @@ __device__ __forceinline__ void load_lane_rows(const __nv_bfloat16* X, const flo
 // the forward's window scores); results land in out_row[d0 .. d0+LC).
 template <int LC, bool F16>
 __device__ __forceinline__ void window_dots(const uint4* ring, int RB, int ig, int d0, int c,
-                                            const float (&q)[4][16], float* out_row) {
+                                            const float (&q)[4][16], float* out_row,
+                                            int i_own, float* mx) {
   float acc[4][LC];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
@@ -114,7 +128,10 @@ __device__ __forceinline__ void window_dots(const uint4* ring, int RB, int ig, i
   float out[LC];
   reduce_scatter4<LC>(acc, out, c);
 #pragma unroll
-  for (int l = 0; l < LC; ++l) out_row[d0 + l] = out[l];
+  for (int l = 0; l < LC; ++l) {
+    out_row[d0 + l] = out[l];
+    if (mx && i_own - (d0 + l) >= 0) *mx = fmaxf(*mx, out[l]);
+  }
 }
 
 // o[q] += w[q][lag] * ring row, over lags [d0, d0+LC) (weights per query row).
@@ -156,7 +173,7 @@ __device__ __forceinline__ void member_dots(const FastBwdArgs& a, uint4* ring, u
                                             const __nv_bfloat16* src, const OffGeo* sg,
                                             const int* s_fold, int i0, int ig, int c, int S_rows,
                                             const float (&x)[4][16], float* val_row,
-                                            float* diff_row) {
+                                            float* diff_row, int i_own, float* mx) {
   constexpr int M = kFastM;
   const int T = a.T, W = a.W, S = a.S, RB = a.ring_rows;
   const int win_lo = max(0, i0 - W + 1), win_hi = min(T, i0 + M);
@@ -164,7 +181,7 @@ __device__ __forceinline__ void member_dots(const FastBwdArgs& a, uint4* ring, u
   stage_rows<ROT>(ring, RB, src, a.rope, win_lo, win_hi);
   stage_sinks<ROT>(sinkb, S_rows, src, a.rope);
   __syncthreads();
-#define SA_CALL(LC) window_dots<LC, ROT>(ring, RB, ig, d0, c, x, val_row)
+#define SA_CALL(LC) window_dots<LC, ROT>(ring, RB, ig, d0, c, x, val_row, i_own, mx)
   SA_WINDOW_CHUNKS(W, SA_CALL)
 #undef SA_CALL
   for (int s0 = 0; s0 < S; s0 += 4) {
@@ -180,19 +197,30 @@ __device__ __forceinline__ void member_dots(const FastBwdArgs& a, uint4* ring, u
     reduce_scatter4<4>(acc, out, c);
 #pragma unroll
     for (int j = 0; j < 4; ++j)
-      if (s0 + j < S) val_row[W + s0 + j] = out[j];
+      if (s0 + j < S) {
+        val_row[W + s0 + j] = out[j];
+        if (mx && s0 + j <= i_own) *mx = fmaxf(*mx, out[j]);
+      }
   }
+  // far offsets, staged in batches whose rows span at most RB rows
   int low = win_lo;
-  for (int kk = 0; kk < a.n_off; ++kk) {
-    if (s_fold[kk]) continue;
-    const OffGeo g = sg[kk];
-    const int seg_lo = max(0, i0 - g.lo - 1), seg_hi = min(T, i0 + M - g.lo);
-    if (seg_lo < low && seg_lo < seg_hi) {
+  int kb = next_far(s_fold, -1, a.n_off);
+  while (kb < a.n_off) {
+    const int hi = qseg_hi(sg[kb], i0, T);
+    int last = kb, nx = next_far(s_fold, kb, a.n_off);
+    while (nx < a.n_off && hi - qseg_lo(sg[nx], i0) <= RB) {
+      last = nx;
+      nx = next_far(s_fold, nx, a.n_off);
+    }
+    const int lo_row = qseg_lo(sg[last], i0);
+    if (lo_row < low && lo_row < hi) {
       __syncthreads();
-      stage_rows<ROT>(ring, RB, src, a.rope, seg_lo, min(seg_hi, low));
-      low = seg_lo;
+      stage_rows<ROT>(ring, RB, src, a.rope, lo_row, min(hi, low));
+      low = lo_row;
       __syncthreads();
     }
+    for (int kk = kb; kk < nx; kk = next_far(s_fold, kk, a.n_off)) {
+    const OffGeo g = sg[kk];
     float pa[4], pb[4];
 #pragma unroll
     for (int u = 0; u < 5; ++u) {
@@ -212,6 +240,9 @@ __device__ __forceinline__ void member_dots(const FastBwdArgs& a, uint4* ring, u
     reduce_scatter4<2>(part, out, c);
     val_row[W + S + kk] = out[0];
     diff_row[kk] = out[1];
+    if (mx && i_own - g.c >= 0) *mx = fmaxf(*mx, out[0]);
+    }
+    kb = nx;
   }
 }
 
@@ -272,10 +303,12 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
   float x[4][16];
   // pass 1: scores and row-score differences (K ring)
   load_lane_rows<true>(Q, a.rope, ig, T, c, a.scale * kKeyUnstage, x);
-  member_dots<true>(a, ring, sinkb, K, sg, s_fold, i0, ig, c, S_rows, x, my_sc, my_dt);
+  float mx = -INFINITY;     // running max of this lane's query's valid scores
+  member_dots<true>(a, ring, sinkb, K, sg, s_fold, i0, ig, c, S_rows, x, my_sc, my_dt, ig + c, &mx);
   // pass 2: dO . values and value differences (V ring)
   load_lane_rows<false>(dO, a.rope, ig, T, c, 1.f, x);
-  member_dots<false>(a, ring, sinkb, V, sg, s_fold, i0, ig, c, S_rows, x, my_dp, my_dpi);
+  member_dots<false>(a, ring, sinkb, V, sg, s_fold, i0, ig, c, S_rows, x, my_dp, my_dpi, ig + c,
+                     nullptr);
   __syncthreads();
 
   // owner lane: probabilities, D_i, dsigma, d-alpha, folded window weights
@@ -295,31 +328,26 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
       }
       // softmax normalised from these scores (not the forward's LSE), so
       // that sum_m p_m = 1 and sum_m g_m = 0 hold for the values used here
-      auto valid = [&](int m) {
-        if (m < W) return i - m >= 0;
-        if (m < W + S) return m - W <= i;
-        return i - sg[m - W - S].c >= 0;
-      };
-      float mx = -INFINITY;
-      for (int m = 0; m < n_slot; ++m) if (valid(m)) mx = fmaxf(mx, my_sc[m]);
-      float l = 0.f;
+      for (int kk = 0; kk < n_off; ++kk)      // near offsets join the running max
+        if (s_fold[kk] && i - sg[kk].c >= 0) mx = fmaxf(mx, my_sc[W + S + kk]);
+      float l = 0.f, edp = 0.f;
       for (int m = 0; m < n_slot; ++m) {
-        const float e = valid(m) ? __expf(my_sc[m] - mx) : 0.f;
+        bool valid;
+        if (m < W) valid = i - m >= 0;
+        else if (m < W + S) valid = m - W <= i;
+        else valid = i - sg[m - W - S].c >= 0;
+        const float e = valid ? __expf(my_sc[m] - mx) : 0.f;
         my_sc[m] = e;
         l += e;
+        edp += e * my_dp[m];
       }
       const float inv = 1.f / l;
-      float Dsum = 0.f;
+      const float Dsum = edp * inv;
       for (int m = 0; m < n_slot; ++m) {
         const float p = my_sc[m] * inv;
-        Dsum += p * my_dp[m];
-        my_sc[m] = p;                       // sc: sigma -> p (for now)
-      }
-      for (int m = 0; m < n_slot; ++m) {
-        const float p = my_sc[m];
         const float g = p * (my_dp[m] - Dsum);
         my_dp[m] = p;                       // dp -> p
-        my_sc[m] = g;                       // sc -> g
+        my_sc[m] = g;                       // sc -> g (dsigma)
       }
       for (int kk = 0; kk < n_off; ++kk) {
         const OffGeo g = sg[kk];
@@ -371,29 +399,38 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
       for (int qq = 0; qq < 4; ++qq) axpy16(x[qq], grp_sc[qq * st + W + s], y);
     }
     int low = win_lo;
-    for (int kk = 0; kk < n_off; ++kk) {
-      if (s_fold[kk]) continue;
-      const OffGeo g = sg[kk];
-      const int two = g.w != 0.f;
-      const int seg_lo = max(0, i0 - g.lo - 1), seg_hi = min(T, i0 + M - g.lo);
-      if (seg_lo < low && seg_lo < seg_hi) {
+    int kb = next_far(s_fold, -1, n_off);
+    while (kb < n_off) {
+      const int hi = qseg_hi(sg[kb], i0, T);
+      int last = kb, nx = next_far(s_fold, kb, n_off);
+      while (nx < n_off && hi - qseg_lo(sg[nx], i0) <= RB) {
+        last = nx;
+        nx = next_far(s_fold, nx, n_off);
+      }
+      const int lo_row = qseg_lo(sg[last], i0);
+      if (lo_row < low && lo_row < hi) {
         __syncthreads();
-        stage_rows<true>(ring, RB, K, a.rope, seg_lo, min(seg_hi, low));
-        low = seg_lo;
+        stage_rows<true>(ring, RB, K, a.rope, lo_row, min(hi, low));
+        low = lo_row;
         __syncthreads();
       }
-      float gq[4];
+      for (int kk = kb; kk < nx; kk = next_far(s_fold, kk, n_off)) {
+        const OffGeo g = sg[kk];
+        const int two = g.w != 0.f;
+        float gq[4];
 #pragma unroll
-      for (int qq = 0; qq < 4; ++qq) gq[qq] = grp_sc[qq * st + W + S + kk];
+        for (int qq = 0; qq < 4; ++qq) gq[qq] = grp_sc[qq * st + W + S + kk];
 #pragma unroll
-      for (int u = 0; u < 5; ++u) {
-        if (u == 0 && !two) continue;
-        const int row = max(ig - g.lo - 1 + u, 0);
-        float y[16];
-        ring_load<true>(ring, row & (RB - 1), c, y);
-        if (u <= 3 && two) axpy16(x[u], gq[u] * g.w, y);
-        if (u >= 1) axpy16(x[u - 1], gq[u - 1] * g.wa, y);
+        for (int u = 0; u < 5; ++u) {
+          if (u == 0 && !two) continue;
+          const int row = max(ig - g.lo - 1 + u, 0);
+          float y[16];
+          ring_load<true>(ring, row & (RB - 1), c, y);
+          if (u <= 3 && two) axpy16(x[u], gq[u] * g.w, y);
+          if (u >= 1) axpy16(x[u - 1], gq[u - 1] * g.wa, y);
+        }
       }
+      kb = nx;
     }
 #pragma unroll
     for (int qq = 0; qq < 4; ++qq) {
@@ -561,26 +598,37 @@ __device__ __forceinline__ void key_pass(const FastBwdArgs& a, uint4* ring, floa
 #undef SA_KEY_WINDOW
     d0 += LCr;
   }
-  // far offsets: query rg+lo+u is row a of key rg+u and row b of key rg+u-1
-  for (int kk = 0; kk < a.n_off; ++kk) {
-    if (s_fold[kk]) continue;
-    const OffGeo g = sg[kk];
-    const int seg_lo = r0 + g.lo, seg_hi = r0 + M + g.lo + 1;
-    if (seg_hi > high) {
+  // far offsets: query rg+lo+u is row a of key rg+u and row b of key rg+u-1.
+  // Member kk needs query rows [r0+lo, r0+M+lo+1); consecutive members whose
+  // rows span at most RB rows are staged in one round.
+  int kb = next_far(s_fold, -1, a.n_off);
+  while (kb < a.n_off) {
+    const int lo_first = r0 + sg[kb].lo;
+    int last = kb, nx = next_far(s_fold, kb, a.n_off);
+    while (nx < a.n_off && r0 + M + sg[nx].lo + 1 - lo_first <= RB) {
+      last = nx;
+      nx = next_far(s_fold, nx, a.n_off);
+    }
+    const int hi_last = r0 + M + sg[last].lo + 1;
+    if (hi_last > high) {
       __syncthreads();
-      stage_sources<ROT>(a, ring, wring, src, wsrc, max(seg_lo, high), seg_hi);
-      high = seg_hi;
+      stage_sources<ROT>(a, ring, wring, src, wsrc, max(lo_first, high), hi_last);
+      high = hi_last;
       __syncthreads();
     }
+    for (int kk = kb; kk < nx; kk = next_far(s_fold, kk, a.n_off)) {
+      const OffGeo g = sg[kk];
 #pragma unroll
-    for (int u = 0; u < 5; ++u) {
-      const int slot = (rg + g.lo + u) & (RB - 1);
-      float y[16];
-      ring_load(ring, slot, c, y);
-      const float gk = wring[slot * wp + W + kk];
-      if (u <= 3) axpy16(d[u], g.wa * gk, y);
-      if (u >= 1) axpy16(d[u - 1], g.w * gk, y);
+      for (int u = 0; u < 5; ++u) {
+        const int slot = (rg + g.lo + u) & (RB - 1);
+        float y[16];
+        ring_load(ring, slot, c, y);
+        const float gk = wring[slot * wp + W + kk];
+        if (u <= 3) axpy16(d[u], g.wa * gk, y);
+        if (u >= 1) axpy16(d[u - 1], g.w * gk, y);
+      }
     }
+    kb = nx;
   }
 }
 
