@@ -108,7 +108,7 @@ __device__ __forceinline__ int next_far(const int* s_fold, int k, int n_off) {
   return k;
 }
 
-__global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
+__global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
   constexpr int M = kFastM;
   extern __shared__ __align__(16) unsigned char smem[];
   uint4* ring = reinterpret_cast<uint4*>(smem);
@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
 
   // ---------------- pass 1: scores ----------------
   __syncthreads();
-  stage_rows<true>(ring, RB, K, a.rope, win_lo, win_hi);
+  stage_rotate<true>(ring, RB, K, a.rope, win_lo, win_hi, kKeyStage);
   stage_sinks<true>(sinkb, S_rows, K, a.rope);
   __syncthreads();
   {
@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
       const int lo_row = far_seg_lo(sg[last], i0);
       if (lo_row < low && lo_row < hi) {
         __syncthreads();
-        stage_rows<true>(ring, RB, K, a.rope, lo_row, min(hi, low));
+        stage_rotate<true>(ring, RB, K, a.rope, lo_row, min(hi, low), kKeyStage);
         low = lo_row;
         __syncthreads();
       }
@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
 #pragma unroll
     for (int h = 0; h < 16; ++h) o[qq][h] = 0.f;
   const float* grp_sc = sc + (size_t)(4 * gid) * a.sc_stride;
-  stage_rows<false>(ring, RB, V, a.rope, win_lo, win_hi);
+  stage_copy(ring, RB, V, win_lo, win_hi);
   stage_sinks<false>(sinkb, S_rows, V, a.rope);
   __syncthreads();
   {
@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(kFastM) k_fwd_fast(const FastArgs a) {
       const int lo_row = far_seg_lo(sg[last], i0);
       if (lo_row < low && lo_row < hi) {
         __syncthreads();
-        stage_rows<false>(ring, RB, V, a.rope, lo_row, min(hi, low));
+        stage_copy(ring, RB, V, lo_row, min(hi, low));
         low = lo_row;
         __syncthreads();
       }

@@ -145,6 +145,97 @@ __device__ __forceinline__ void stage_rows(uint4* ring, int ring_rows, const __n
   }
 }
 
+// Asynchronous 16-byte global -> shared copy (completes at cp_async_wait_all).
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
+}
+
+// Copy rows [a, b) of a bf16 [T][64] array into ring slots row & (ring_rows-1),
+// every 16-byte chunk in flight at once (all rows here are < T).  The caller
+// synchronises the CTA afterwards.
+__device__ __forceinline__ void stage_copy(uint4* ring, int ring_rows, const __nv_bfloat16* src,
+                                           int a, int b) {
+  const int n = (b - a) * kChunks;
+  for (int task = threadIdx.x; task < n; task += blockDim.x) {
+    const int row = a + (task >> 3), ch = task & 7;
+    const int slot = row & (ring_rows - 1);
+    cp_async16(ring + slot * kChunks + (ch ^ swz(slot)),
+               reinterpret_cast<const uint4*>(src + (size_t)row * kD) + ch);
+  }
+  cp_async_wait_all();
+}
+
+// Stage rows [a, b) (all < T) rotated by RoPE at their own positions, times
+// `mul`, as fp16 (OUT_F16: keys) or bf16 (queries).  Every raw row chunk is
+// first copied asynchronously into its ring slot; meanwhile each thread loads
+// the cos/sin of the first row of its run and the per-row angle step theta_j
+// (table row 1) for its RoPE pair-chunk p; after the copies land (one CTA
+// barrier) each thread rotates its run of consecutive rows in place, stepping
+// the angle by theta_j per row (a run is at most a few rows, so the fp32
+// recurrence stays within ~1e-6 of the table).  The caller synchronises after.
+template <bool OUT_F16>
+__device__ __forceinline__ void stage_rotate(uint4* ring, int ring_rows, const __nv_bfloat16* src,
+                                             const float2* rope, int a, int b, float mul) {
+  const int n = b - a;
+  if (n <= 0) return;
+  for (int task = threadIdx.x; task < n * kChunks; task += blockDim.x) {
+    const int row = a + (task >> 3), ch = task & 7;
+    const int slot = row & (ring_rows - 1);
+    cp_async16(ring + slot * kChunks + (ch ^ swz(slot)),
+               reinterpret_cast<const uint4*>(src + (size_t)row * kD) + ch);
+  }
+  const int runs = blockDim.x >> 2;
+  const int L = (n + runs - 1) / runs;
+  const int p = threadIdx.x & 3;
+  const int r0 = a + (int)(threadIdx.x >> 2) * L;
+  const int r1 = min(r0 + L, b);
+  float2 cs[8];
+  if (r0 < r1) {
+    const float4* g0 = reinterpret_cast<const float4*>(rope + (size_t)r0 * 32 + 8 * p);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float4 u = __ldg(g0 + h);
+      cs[2 * h] = make_float2(u.x, u.y); cs[2 * h + 1] = make_float2(u.z, u.w);
+    }
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  if (r0 >= r1) return;
+  float2 st[8];      // the same table row for every run: cached after first use
+  {
+    const float4* g1 = reinterpret_cast<const float4*>(rope + 32 + 8 * p);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float4 w = __ldg(g1 + h);
+      st[2 * h] = make_float2(w.x, w.y); st[2 * h + 1] = make_float2(w.z, w.w);
+    }
+  }
+  for (int row = r0; row < r1; ++row) {
+    const int slot = row & (ring_rows - 1);
+    const int sw = swz(slot);
+    uint4* c0 = ring + slot * kChunks + (p ^ sw);
+    uint4* c1 = ring + slot * kChunks + ((p + 4) ^ sw);
+    float x1[8], x2[8];
+    unpack8(*c0, x1);
+    unpack8(*c1, x2);
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      const float a0 = x1[h], b0 = x2[h];
+      x1[h] = (a0 * cs[h].x - b0 * cs[h].y) * mul;
+      x2[h] = (b0 * cs[h].x + a0 * cs[h].y) * mul;
+      const float c2 = cs[h].x * st[h].x - cs[h].y * st[h].y;
+      cs[h].y = cs[h].y * st[h].x + cs[h].x * st[h].y;
+      cs[h].x = c2;
+    }
+    *c0 = OUT_F16 ? pack8_h(x1) : pack8(x1);
+    *c1 = OUT_F16 ? pack8_h(x2) : pack8(x2);
+  }
+}
+
 // Sink rows 0..S-1 into a plain (unswizzled) buffer.
 template <bool ROT>
 __device__ __forceinline__ void stage_sinks(uint4* buf, int S, const __nv_bfloat16* src,
