@@ -97,7 +97,9 @@ size_t sparse_attn_workspace_size(const sa_params* p, int backward);
  *   o       : device [L][B][H][T][D], dtype p->dtype            (written)
  *   lse     : device fp32 [L][B][H][T] or NULL                  (written)
  *   workspace / workspace_bytes: device scratch of at least
- *             sparse_attn_workspace_size(p, 0) bytes (may be NULL if 0).
+ *             sparse_attn_workspace_size(p, 0) bytes, 16-byte aligned (may be
+ *             NULL if 0).  The bf16 / D = 64 path keeps the RoPE-rotated keys
+ *             there (L*B*H*T*D 16-bit values); other configurations need none.
  * Source: "Depth-Staggered Fibonacci Spacing for Sparse Attention",
  * Methodology -- "Attended set", "Scaling", "Implementation".
  */
@@ -153,6 +155,14 @@ sa_status sparse_attn_bwd(const sa_params* p, const void* q, const void* k, cons
 sa_status sparse_attn_fwd_noalloc(const sa_params* p, const void* q, const void* k,
                                   const void* v, const float* alpha, void* o, float* lse,
                                   void* stream);
+
+/*
+ * Device error word of the staged kernels: bit 0 is set when a bounded wait
+ * for a staging copy gave up (the kernel then left its outputs incomplete and
+ * returned rather than wait without end).  Reading synchronises with the
+ * device; with clear != 0 the word is reset.  Returns -1 on a CUDA error.
+ */
+int32_t sparse_attn_device_error(int clear);
 
 /* Static, NUL-terminated description of a status code. */
 const char* sparse_attn_status_string(sa_status s);

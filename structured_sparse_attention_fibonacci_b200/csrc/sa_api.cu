@@ -107,8 +107,9 @@ sa_status validate_params(const sa_params* p, Problem* pb) { return build_proble
 
 cudaError_t launch_fwd_dispatch(const Problem& pb, const FwdPtrs& a, cudaStream_t st,
                                 int* launches) {
-  return (!g_force_general && fast_fwd_supported(pb)) ? launch_fwd_fast(pb, a, st, launches)
-                                                      : launch_fwd_general(pb, a, st, launches);
+  return (!g_force_general && fast_fwd_supported(pb))
+             ? launch_fwd_fast(pb, a, nullptr, st, launches)
+             : launch_fwd_general(pb, a, st, launches);
 }
 
 void trace_mark(const char* kernel, cudaStream_t st, bool begin) {
@@ -179,10 +180,16 @@ int32_t sparse_attn_trace_read(int32_t max, const char** names, double* total_ms
   return (int32_t)nm.size();
 }
 
+int32_t sparse_attn_device_error(int clear) {
+  unsigned fwd = 0;
+  if (sa::fast_fwd_read_error(&fwd, clear != 0) != cudaSuccess) return -1;
+  return (int32_t)fwd;
+}
+
 size_t sparse_attn_workspace_size(const sa_params* p, int backward) {
   sa::Problem pb;
   if (build_problem(p, &pb) != SA_OK) return 0;
-  if (!backward) return 0;
+  if (!backward) return sa::fast_fwd_workspace(pb);
   // enough for whichever backward path a call takes (see sparse_attn_force_general)
   size_t need = sa::general_bwd_layout(pb).total;
   if (sa::fast_bwd_supported(pb)) need = std::max(need, sa::fast_bwd_workspace(pb));
@@ -199,15 +206,16 @@ sa_status sparse_attn_fwd(const sa_params* p, const void* q, const void* k, cons
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (lse && !aligned4(lse)) || !aligned4(alpha))
     return SA_ERR_INVALID_ARG;
-  if (workspace_bytes < sparse_attn_workspace_size(p, 0)) return SA_ERR_WORKSPACE;
-  (void)workspace;
+  const size_t need = sparse_attn_workspace_size(p, 0);
+  if (workspace_bytes < need || (need && (!workspace || !aligned16(workspace))))
+    return SA_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const float2* rope = nullptr;
   if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
   sa::FwdPtrs a = {q, k, v, alpha, o, lse, rope};
   int launches = 0;
   cudaError_t e = (!g_force_general && sa::fast_fwd_supported(pb))
-                      ? sa::launch_fwd_fast(pb, a, st, &launches)
+                      ? sa::launch_fwd_fast(pb, a, workspace, st, &launches)
                       : sa::launch_fwd_general(pb, a, st, &launches);
   if (e != cudaSuccess) return SA_ERR_CUDA;
   g_last_launches = launches;

@@ -4,59 +4,67 @@
 //
 // One CTA owns a tile of M consecutive queries of one (layer, batch, head).
 //  * Lane mapping: a group of 4 lanes owns 4 consecutive queries; lane c of
-//    the group holds dims [8c, 8c+8) and [32+8c, 32+8c+8) of each (a rotate-
-//    half RoPE pair stays in one lane).  Every staged row chunk a lane reads
-//    is reused for up to 4 queries (window) or 2 queries (an interpolated
-//    offset), which keeps shared-memory traffic near one byte per FMA.
+//    the group holds 16 of the 64 dims of each, chunks c and c + 4 (a rotate-
+//    half RoPE pair stays in one lane), in the group-parity order of the ring
+//    reads (sa_stage.cuh).  Every staged row chunk a lane reads is reused for
+//    up to 4 queries (window) or 2 queries (an interpolated offset).
 //  * Partial dot products of the 4 lanes are combined by a 4-lane transpose
 //    reduce-scatter, after which each lane owns one query's full scores.
 //  * Staging: the tile's members are visited in increasing lag order (window,
 //    then the offsets sorted by f).  Each member needs a contiguous row range;
-//    only rows below everything staged so far are fetched, into a ring of
-//    shared-memory rows, so every row of the tile's union is read from L2 once
-//    per pass.  K rows are rotated (RoPE) on the way in and kept as scaled
-//    fp16, V rows as bf16, with a 16-byte-chunk XOR swizzle.
+//    only rows below everything staged so far are fetched, by bulk copies into
+//    a ring of shared-memory rows, so every row of the tile's union is read
+//    from L2 once per pass.  Keys arrive already rotated (fp16 of RoPE(K) /
+//    256, written by the RoPE pre-pass); the allocation-free entry point,
+//    which has no room for that, copies raw K rows and rotates them in place.
 //  * An offset whose rows lie inside the window ("near") costs nothing: its
 //    score is the interpolation of two window scores, and its probability is
-//    folded into the two window weights used for PV.
-//  * Two passes over the members: scores (K ring), softmax by the owner lane,
-//    then PV (V ring).
+//    folded into the two window weights used for PV.  An offset that no query
+//    of the tile has yet ("dead") is skipped.
+//  * Two passes over the members: scores (key ring), softmax by the owner
+//    lane, then PV (value ring).
 #include <algorithm>
 
-#include "sa_fast_common.cuh"
+#include "sa_stage.cuh"
 
 namespace sa {
 
 namespace {
 
 using namespace fast;
+using namespace stage;
 
 struct FastArgs {
   int B, H, T, W, n_off, S, n_tiles;
   int ring_rows, sc_stride;
   float scale;
   int f[SA_MAX_OFFSETS];               // ascending
-  const __nv_bfloat16* q; const __nv_bfloat16* k; const __nv_bfloat16* v;
+  const __nv_bfloat16* q;
+  const void* k;                       // rotated fp16 keys, or raw bf16 K (in-place rotation)
+  const __nv_bfloat16* v;
   const float* alpha; const float2* rope;
   __nv_bfloat16* o; float* lse;
+  unsigned* err;
 };
 
-// Window scores for lags [d0, d0 + LC): rows ig+3-d0-u, u = 0..LC+2; query q
-// (row ig+q) takes row u at lag d0 + (q + u - 3).
+enum : int { kFar = 0, kNear = 1, kDead = 2 };
+
+// Window scores for lags [d0, d0 + LC): rows ig+3-d0-u, u = 0..LC+2, walked
+// upward from the lowest; query q (row ig+q) takes row u at lag d0 + q + u - 3.
 template <int LC>
-__device__ __forceinline__ void window_scores(const uint4* ring, int ring_rows, int ig, int d0,
-                                              int c, const float (&q)[4][16], float* sc_row,
-                                              int i_own, float& mx) {
+__device__ __forceinline__ void window_scores(const unsigned char* ring, int RB, int ig, int d0,
+                                              int off0, int d1, int c, const float (&q)[4][16],
+                                              float* sc_row, int i_own, float& mx) {
   float acc[4][LC];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int l = 0; l < LC; ++l) acc[a][l] = 0.f;
+  const unsigned char* p = ring + (size_t)((ig + 1 - d0 - LC) & (RB - 1)) * kRowBytes + off0;
 #pragma unroll
   for (int u = 0; u < LC + 3; ++u) {
-    const int row = max(ig + 3 - d0 - u, 0);
     float x[16];
-    ring_load<true>(ring, row & (ring_rows - 1), c, x);
+    lane_row<true>(p + (LC + 2 - u) * kRowBytes, d1, x);
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int l = a + u - 3;
@@ -74,18 +82,19 @@ __device__ __forceinline__ void window_scores(const uint4* ring, int ring_rows, 
 
 // Window PV for lags [d0, d0 + LC) with weights sc[query][lag].
 template <int LC>
-__device__ __forceinline__ void window_pv(const uint4* ring, int ring_rows, int ig, int d0, int c,
-                                          const float* sc, int stride, float (&o)[4][16]) {
+__device__ __forceinline__ void window_pv(const unsigned char* ring, int RB, int ig, int d0,
+                                          int off0, int d1, const float* sc, int stride,
+                                          float (&o)[4][16]) {
   float pw[4][LC];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int l = 0; l < LC; ++l) pw[a][l] = sc[a * stride + d0 + l];
+  const unsigned char* p = ring + (size_t)((ig + 1 - d0 - LC) & (RB - 1)) * kRowBytes + off0;
 #pragma unroll
   for (int u = 0; u < LC + 3; ++u) {
-    const int row = max(ig + 3 - d0 - u, 0);
     float x[16];
-    ring_load(ring, row & (ring_rows - 1), c, x);
+    lane_row<false>(p + (LC + 2 - u) * kRowBytes, d1, x);
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int l = a + u - 3;
@@ -94,46 +103,118 @@ __device__ __forceinline__ void window_pv(const uint4* ring, int ring_rows, int 
   }
 }
 
-// Rows a far offset's member needs for the tile [i0, i0 + M): [lo, hi).
-__device__ __forceinline__ int far_seg_lo(const OffGeo& g, int i0) {
-  return max(0, i0 - g.lo - (g.w != 0.f ? 1 : 0));
-}
-__device__ __forceinline__ int far_seg_hi(const OffGeo& g, int i0, int T) {
-  return max(0, min(T, i0 + kFastM - g.lo));
-}
-// Next offset after k that is not folded into the window (n_off when none).
-__device__ __forceinline__ int next_far(const int* s_fold, int k, int n_off) {
+// Next offset after k that is neither near nor dead (n_off when none).
+__device__ __forceinline__ int next_far(const int* s_kind, int k, int n_off) {
   ++k;
-  while (k < n_off && s_fold[k]) ++k;
+  while (k < n_off && s_kind[k] != kFar) ++k;
   return k;
 }
 
+// Rotate, in place, the raw bf16 K rows [a, b) (all inside [0, T)) staged in
+// the ring (RB > 0) or in a plain buffer (RB == 0, row r at r * 128), into
+// fp16 of RoPE(K) * kKeyStage.  Thread (run j, pair-chunk p) walks a run of
+// consecutive rows, stepping the angles by theta_j per row (a run is a few
+// rows, so the fp32 recurrence stays within ~1e-6 of the table); odd runs
+// touch their two chunks in the opposite order (bank-conflict-free).
+__device__ __forceinline__ void rotate_rows(unsigned char* buf, int RB, const float2* rope, int a,
+                                            int b) {
+  const int n = b - a;
+  if (n <= 0) return;
+  const int runs = blockDim.x >> 2;
+  const int L = (n + runs - 1) / runs;
+  const int j = threadIdx.x >> 2, p = threadIdx.x & 3, par = j & 1;
+  const int r0 = a + j * L, r1 = min(r0 + L, b);
+  if (r0 >= r1) return;
+  float2 cs[8], st[8];
+  {
+    const float4* g0 = reinterpret_cast<const float4*>(rope + (size_t)r0 * 32 + 8 * p);
+    const float4* g1 = reinterpret_cast<const float4*>(rope + 32 + 8 * p);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float4 u = __ldg(g0 + h), w = __ldg(g1 + h);
+      cs[2 * h] = make_float2(u.x, u.y); cs[2 * h + 1] = make_float2(u.z, u.w);
+      st[2 * h] = make_float2(w.x, w.y); st[2 * h + 1] = make_float2(w.z, w.w);
+    }
+  }
+  const int o0 = half0_off(p, par), o1 = half1_off(p, par);
+  for (int row = r0; row < r1; ++row) {
+    const int slot = RB ? (row & (RB - 1)) : row;
+    uint4* c0 = reinterpret_cast<uint4*>(buf + (size_t)slot * kRowBytes + o0);
+    uint4* c1 = reinterpret_cast<uint4*>(buf + (size_t)slot * kRowBytes + o1);
+    float y0[8], y1[8];
+    unpack8(*c0, y0);
+    unpack8(*c1, y1);
+    float x1[8], x2[8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      const float lo = par ? y1[h] : y0[h], hi = par ? y0[h] : y1[h];
+      x1[h] = (lo * cs[h].x - hi * cs[h].y) * kKeyStage;
+      x2[h] = (hi * cs[h].x + lo * cs[h].y) * kKeyStage;
+      const float c2 = cs[h].x * st[h].x - cs[h].y * st[h].y;
+      cs[h].y = cs[h].y * st[h].x + cs[h].x * st[h].y;
+      cs[h].x = c2;
+    }
+    const uint4 u1 = pack8_h(x1), u2 = pack8_h(x2);
+    *c0 = par ? u2 : u1;
+    *c1 = par ? u1 : u2;
+    if (RB && slot < kMirror) {
+      *reinterpret_cast<uint4*>(buf + (size_t)(RB + slot) * kRowBytes + o0) = par ? u2 : u1;
+      *reinterpret_cast<uint4*>(buf + (size_t)(RB + slot) * kRowBytes + o1) = par ? u1 : u2;
+    }
+  }
+}
+
+// One staging round of key rows [a, b) into the ring (plus, on the first
+// round, the sink rows): copies, wait, and for raw keys the in-place rotation.
+// Returns nonzero when a wait gave up (the kernel then returns).
+template <bool PRE>
+__device__ __forceinline__ int stage_keys(Stager& s, unsigned char* ring, int RB,
+                                          unsigned char* sinkb, const FastArgs& a,
+                                          const unsigned char* K, int S_stage, int T, int lo,
+                                          int hi) {
+  stage_ring(s, ring, RB, K, T, lo, hi);
+  if (S_stage) stage_plain(s, sinkb, K, min(a.S, T), a.S);
+  if (stage_commit_wait(s)) { stage_drain(s); return 1; }
+  if (!PRE) {
+    rotate_rows(ring, RB, a.rope, max(lo, 0), min(hi, T));
+    if (S_stage) rotate_rows(sinkb, 0, a.rope, 0, min(a.S, T));
+    __syncthreads();
+  }
+  return 0;
+}
+
+template <bool PRE>
 __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
   constexpr int M = kFastM;
-  extern __shared__ __align__(16) unsigned char smem[];
-  uint4* ring = reinterpret_cast<uint4*>(smem);
-  uint4* sinkb = ring + (size_t)a.ring_rows * kChunks;
-  float* sc = reinterpret_cast<float*>(sinkb + (size_t)a.S * kChunks);
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int RB = a.ring_rows;
+  unsigned char* ring = smem;
+  unsigned char* sinkb = smem + (size_t)(RB + kMirror) * kRowBytes;
+  float* sc = reinterpret_cast<float*>(sinkb + (size_t)a.S * kRowBytes);
   __shared__ OffGeo sg[SA_MAX_OFFSETS];
-  __shared__ int s_fold[SA_MAX_OFFSETS];
+  __shared__ int s_kind[SA_MAX_OFFSETS];
+  __shared__ uint64_t bar;
 
   const int unit = blockIdx.x / a.n_tiles, tile = blockIdx.x % a.n_tiles;
   const int layer = unit / (a.B * a.H);
   const int T = a.T, W = a.W, S = a.S, n_off = a.n_off;
   const int i0 = tile * M;
-  const int t = threadIdx.x, gid = t >> 2, c = t & 3;
+  const int t = threadIdx.x, gid = t >> 2, c = t & 3, par = gid & 1;
   const int ig = i0 + 4 * gid;
   const size_t ub = (size_t)unit * T * kD;
   const __nv_bfloat16* Q = a.q + ub;
-  const __nv_bfloat16* K = a.k + ub;
-  const __nv_bfloat16* V = a.v + ub;
+  const unsigned char* K = reinterpret_cast<const unsigned char*>(a.k) + ub * 2;
+  const unsigned char* V = reinterpret_cast<const unsigned char*>(a.v + ub);
 
+  if (t == 0) { mbar_init(&bar, 1); fence_barrier_init(); }
   int bad = 0;
   if (t < n_off) {
     const OffGeo g = offset_geometry(__ldg(a.alpha + layer), a.f[t]);
     sg[t] = g;
     bad = !g.ok;
-    s_fold[t] = g.ok && (g.lo + (g.w != 0.f ? 1 : 0) <= W - 1);
+    const int near = g.ok && (g.lo + (g.w != 0.f ? 1 : 0) <= W - 1);
+    const int dead = i0 + M - 1 - g.c < 0;        // no query of the tile has it yet
+    s_kind[t] = near ? kNear : (dead ? kDead : kFar);
   }
   bad = __syncthreads_or(bad);
   if (bad) {  // the layer has an offset with no defined row: NaN outputs
@@ -150,14 +231,10 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
     }
     return;
   }
+  Stager stg{&bar, 0u, a.err};
 
-  // zero the ring and the sink rows so unstaged slots always hold finite values
-  // (sink rows s >= T are never attended and never staged)
-  for (int e = t; e < (a.ring_rows + S) * kChunks; e += M) ring[e] = make_uint4(0, 0, 0, 0);
-  const int S_rows = min(S, T);
-
-  // this lane's slice of its 4 queries, rotated and scaled (times the inverse
-  // of the key staging factor)
+  // This lane's slice of its 4 queries, rotated and scaled (times the inverse
+  // of the key staging factor), first half = chunk c + 4 * par.
   const float qs = a.scale * kKeyUnstage;
   float q[4][16];
 #pragma unroll
@@ -171,38 +248,39 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
 #pragma unroll
     for (int h = 0; h < 8; h += 2) {
       const float4 tt = __ldg(cs + h / 2);
-      q[qq][h] = (x1[h] * tt.x - x2[h] * tt.y) * qs;
-      q[qq][h + 8] = (x2[h] * tt.x + x1[h] * tt.y) * qs;
-      q[qq][h + 1] = (x1[h + 1] * tt.z - x2[h + 1] * tt.w) * qs;
-      q[qq][h + 9] = (x2[h + 1] * tt.z + x1[h + 1] * tt.w) * qs;
+      const float r0 = (x1[h] * tt.x - x2[h] * tt.y) * qs;
+      const float r1 = (x2[h] * tt.x + x1[h] * tt.y) * qs;
+      const float r2 = (x1[h + 1] * tt.z - x2[h + 1] * tt.w) * qs;
+      const float r3 = (x2[h + 1] * tt.z + x1[h + 1] * tt.w) * qs;
+      q[qq][h] = par ? r1 : r0;
+      q[qq][h + 8] = par ? r0 : r1;
+      q[qq][h + 1] = par ? r3 : r2;
+      q[qq][h + 9] = par ? r2 : r3;
     }
   }
+  const int off0 = half0_off(c, par), d1 = half1_off(c, par) - off0;
 
   const int lr = 4 * gid + c;                  // this lane's query, tile-local
   const int i_own = ig + c;                    // ... and its position
   float mx = -INFINITY;                        // running max of its valid scores
   float* my_sc = sc + (size_t)lr * a.sc_stride;
-  const int win_lo = max(0, i0 - W + 1), win_hi = min(T, i0 + M);
-  const int RB = a.ring_rows;
+  const int win_lo = i0 - W + 1, win_hi = i0 + M;
 
   // ---------------- pass 1: scores ----------------
-  __syncthreads();
-  stage_rotate<true>(ring, RB, K, a.rope, win_lo, win_hi, kKeyStage);
-  stage_sinks<true>(sinkb, S_rows, K, a.rope);
-  __syncthreads();
+  if (stage_keys<PRE>(stg, ring, RB, sinkb, a, K, 1, T, win_lo, win_hi)) return;
   {
     int d0 = 0;
-    while (W - d0 >= 8) { window_scores<8>(ring, RB, ig, d0, c, q, my_sc, i_own, mx); d0 += 8; }
-    if (W - d0 >= 4) { window_scores<4>(ring, RB, ig, d0, c, q, my_sc, i_own, mx); d0 += 4; }
-    if (W - d0 >= 2) { window_scores<2>(ring, RB, ig, d0, c, q, my_sc, i_own, mx); d0 += 2; }
-    if (W - d0 >= 1) { window_scores<1>(ring, RB, ig, d0, c, q, my_sc, i_own, mx); d0 += 1; }
+    while (W - d0 >= 8) { window_scores<8>(ring, RB, ig, d0, off0, d1, c, q, my_sc, i_own, mx); d0 += 8; }
+    if (W - d0 >= 4) { window_scores<4>(ring, RB, ig, d0, off0, d1, c, q, my_sc, i_own, mx); d0 += 4; }
+    if (W - d0 >= 2) { window_scores<2>(ring, RB, ig, d0, off0, d1, c, q, my_sc, i_own, mx); d0 += 2; }
+    if (W - d0 >= 1) { window_scores<1>(ring, RB, ig, d0, off0, d1, c, q, my_sc, i_own, mx); d0 += 1; }
   }
   for (int s0 = 0; s0 < S; s0 += 4) {
     float acc[4][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       float x[16];
-      sink_load<true>(sinkb, min(s0 + j, S - 1), c, x);
+      lane_row<true>(sinkb + (size_t)min(s0 + j, S - 1) * kRowBytes + off0, d1, x);
 #pragma unroll
       for (int qq = 0; qq < 4; ++qq) acc[qq][j] = dot16(q[qq], x);
     }
@@ -216,35 +294,34 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
       }
   }
   // far offsets, staged in batches: consecutive members whose rows span at
-  // most RB rows share one staging round and are computed back to back
+  // most RB rows share one staging round and are computed back to back.  A
+  // far member reads rows [i0 - lo - 1, i0 + M - lo).
   {
     int low = win_lo;
-    int kk = next_far(s_fold, -1, n_off);
+    int kk = next_far(s_kind, -1, n_off);
     while (kk < n_off) {
-      const int hi = far_seg_hi(sg[kk], i0, T);
-      int last = kk, nx = next_far(s_fold, kk, n_off);
-      while (nx < n_off && hi - far_seg_lo(sg[nx], i0) <= RB) {
+      const int hi = i0 + M - sg[kk].lo;
+      int last = kk, nx = next_far(s_kind, kk, n_off);
+      while (nx < n_off && hi - (i0 - sg[nx].lo - 1) <= RB) {
         last = nx;
-        nx = next_far(s_fold, nx, n_off);
+        nx = next_far(s_kind, nx, n_off);
       }
-      // rows the batch needs: [lo_row, hi); only those below `low` are new
-      const int lo_row = far_seg_lo(sg[last], i0);
-      if (lo_row < low && lo_row < hi) {
+      const int lo_row = i0 - sg[last].lo - 1;
+      if (lo_row < low) {              // only rows below everything staged are new
         __syncthreads();
-        stage_rotate<true>(ring, RB, K, a.rope, lo_row, min(hi, low), kKeyStage);
+        if (stage_keys<PRE>(stg, ring, RB, sinkb, a, K, 0, T, lo_row, min(hi, low))) return;
         low = lo_row;
-        __syncthreads();
       }
-      for (int m = kk; m < nx; m = next_far(s_fold, m, n_off)) {
+      for (int m = kk; m < nx; m = next_far(s_kind, m, n_off)) {
         const OffGeo g = sg[m];
         const int two = g.w != 0.f;
+        const unsigned char* p = ring + (size_t)((ig - g.lo - 1) & (RB - 1)) * kRowBytes + off0;
         float pa[4] = {0.f, 0.f, 0.f, 0.f}, pb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int u = 0; u < 5; ++u) {
           if (u == 0 && !two) continue;
-          const int row = max(ig - g.lo - 1 + u, 0);
           float x[16];
-          ring_load<true>(ring, row & (RB - 1), c, x);
+          lane_row<true>(p + u * kRowBytes, d1, x);
           if (u <= 3) pb[u] = dot16(q[u], x);
           if (u >= 1) pa[u - 1] = dot16(q[u - 1], x);
         }
@@ -269,7 +346,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
     const int i = i_own;
     if (i < T) {
       for (int kk = 0; kk < n_off; ++kk) {    // near offsets: from two window scores
-        if (!s_fold[kk]) continue;
+        if (s_kind[kk] != kNear) continue;
         const OffGeo g = sg[kk];
         float sv = g.wa * my_sc[g.lo];
         if (g.w != 0.f) sv += g.w * my_sc[g.lo + 1];
@@ -289,7 +366,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
         const OffGeo g = sg[kk];
         const float e = (i - g.c >= 0) ? __expf(my_sc[W + S + kk] - mx) : 0.f;
         my_sc[W + S + kk] = e; l += e;
-        if (s_fold[kk]) {                      // fold into the two window weights
+        if (s_kind[kk] == kNear) {             // fold into the two window weights
           my_sc[g.lo] += g.wa * e;
           if (g.w != 0.f) my_sc[g.lo + 1] += g.w * e;
         }
@@ -309,51 +386,51 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
 #pragma unroll
     for (int h = 0; h < 16; ++h) o[qq][h] = 0.f;
   const float* grp_sc = sc + (size_t)(4 * gid) * a.sc_stride;
-  stage_copy(ring, RB, V, win_lo, win_hi);
-  stage_sinks<false>(sinkb, S_rows, V, a.rope);
-  __syncthreads();
+  stage_ring(stg, ring, RB, V, T, win_lo, win_hi);
+  stage_plain(stg, sinkb, V, min(S, T), S);
+  if (stage_commit_wait(stg)) { stage_drain(stg); return; }
   {
     int d0 = 0;
-    while (W - d0 >= 8) { window_pv<8>(ring, RB, ig, d0, c, grp_sc, a.sc_stride, o); d0 += 8; }
-    if (W - d0 >= 4) { window_pv<4>(ring, RB, ig, d0, c, grp_sc, a.sc_stride, o); d0 += 4; }
-    if (W - d0 >= 2) { window_pv<2>(ring, RB, ig, d0, c, grp_sc, a.sc_stride, o); d0 += 2; }
-    if (W - d0 >= 1) { window_pv<1>(ring, RB, ig, d0, c, grp_sc, a.sc_stride, o); d0 += 1; }
+    while (W - d0 >= 8) { window_pv<8>(ring, RB, ig, d0, off0, d1, grp_sc, a.sc_stride, o); d0 += 8; }
+    if (W - d0 >= 4) { window_pv<4>(ring, RB, ig, d0, off0, d1, grp_sc, a.sc_stride, o); d0 += 4; }
+    if (W - d0 >= 2) { window_pv<2>(ring, RB, ig, d0, off0, d1, grp_sc, a.sc_stride, o); d0 += 2; }
+    if (W - d0 >= 1) { window_pv<1>(ring, RB, ig, d0, off0, d1, grp_sc, a.sc_stride, o); d0 += 1; }
   }
   for (int s = 0; s < S; ++s) {
     float x[16];
-    sink_load(sinkb, s, c, x);
+    lane_row<false>(sinkb + (size_t)s * kRowBytes + off0, d1, x);
 #pragma unroll
     for (int qq = 0; qq < 4; ++qq) axpy16(o[qq], grp_sc[qq * a.sc_stride + W + s], x);
   }
   {
     int low = win_lo;
-    int kk = next_far(s_fold, -1, n_off);
+    int kk = next_far(s_kind, -1, n_off);
     while (kk < n_off) {
-      const int hi = far_seg_hi(sg[kk], i0, T);
-      int last = kk, nx = next_far(s_fold, kk, n_off);
-      while (nx < n_off && hi - far_seg_lo(sg[nx], i0) <= RB) {
+      const int hi = i0 + M - sg[kk].lo;
+      int last = kk, nx = next_far(s_kind, kk, n_off);
+      while (nx < n_off && hi - (i0 - sg[nx].lo - 1) <= RB) {
         last = nx;
-        nx = next_far(s_fold, nx, n_off);
+        nx = next_far(s_kind, nx, n_off);
       }
-      const int lo_row = far_seg_lo(sg[last], i0);
-      if (lo_row < low && lo_row < hi) {
+      const int lo_row = i0 - sg[last].lo - 1;
+      if (lo_row < low) {
         __syncthreads();
-        stage_copy(ring, RB, V, lo_row, min(hi, low));
+        stage_ring(stg, ring, RB, V, T, lo_row, min(hi, low));
+        if (stage_commit_wait(stg)) { stage_drain(stg); return; }
         low = lo_row;
-        __syncthreads();
       }
-      for (int m = kk; m < nx; m = next_far(s_fold, m, n_off)) {
+      for (int m = kk; m < nx; m = next_far(s_kind, m, n_off)) {
         const OffGeo g = sg[m];
         const int two = g.w != 0.f;
         float p[4];
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) p[qq] = grp_sc[qq * a.sc_stride + W + S + m];
+        const unsigned char* rp = ring + (size_t)((ig - g.lo - 1) & (RB - 1)) * kRowBytes + off0;
 #pragma unroll
         for (int u = 0; u < 5; ++u) {
           if (u == 0 && !two) continue;
-          const int row = max(ig - g.lo - 1 + u, 0);
           float x[16];
-          ring_load(ring, row & (RB - 1), c, x);
+          lane_row<false>(rp + u * kRowBytes, d1, x);
           if (u <= 3 && two) axpy16(o[u], p[u] * g.w, x);
           if (u >= 1) axpy16(o[u - 1], p[u - 1] * g.wa, x);
         }
@@ -366,20 +443,26 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
   float inv[4];
 #pragma unroll
   for (int qq = 0; qq < 4; ++qq) inv[qq] = __shfl_sync(0xffffffffu, inv_l, (t & 28) + qq);
-#pragma unroll
-  for (int qq = 0; qq < 4; ++qq)
-#pragma unroll
-    for (int h = 0; h < 16; ++h) o[qq][h] *= inv[qq];
-
+  const int h0 = c + 4 * par, h1 = c + 4 - 4 * par;
 #pragma unroll
   for (int qq = 0; qq < 4; ++qq) {
     const int i = ig + qq;
+#pragma unroll
+    for (int h = 0; h < 16; ++h) o[qq][h] *= inv[qq];
     if (i < T) {
       uint4* dst = reinterpret_cast<uint4*>(a.o + ub + (size_t)i * kD);
-      dst[c] = pack8(o[qq]);
-      dst[c + 4] = pack8(o[qq] + 8);
+      dst[h0] = pack8(o[qq]);
+      dst[h1] = pack8(o[qq] + 8);
     }
   }
+}
+
+__device__ unsigned g_fwd_err;   // bit 0: a staging wait gave up
+
+int ring_rows_for(const Problem& pb) {
+  int rr = 32;   // a power of two: ring slots are row & (rr - 1)
+  while (rr < std::max(kFastM + pb.W - 1, kFastM + 2)) rr *= 2;
+  return rr;
 }
 
 }  // namespace
@@ -389,18 +472,23 @@ bool fast_fwd_supported(const Problem& pb) {
 }
 
 size_t fast_fwd_smem(const Problem& pb, int* ring_rows, int* sc_stride) {
-  int rr = 32;   // a power of two: ring slots are row & (rr - 1)
-  while (rr < std::max(kFastM + pb.W - 1, kFastM + 2)) rr *= 2;
+  const int rr = ring_rows_for(pb);
   // odd stride: the 8 lane groups of a warp read rows 4 apart, and the 32
   // owner lanes read 32 consecutive rows, without shared-memory bank conflicts
   const int n_slot = pb.W + pb.S + pb.n_off;
   const int st = n_slot | 1;
   if (ring_rows) *ring_rows = rr;
   if (sc_stride) *sc_stride = st;
-  return (size_t)rr * 128 + (size_t)pb.S * 128 + (size_t)kFastM * st * sizeof(float);
+  return (size_t)(rr + kMirror) * kRowBytes + (size_t)pb.S * kRowBytes +
+         (size_t)kFastM * st * sizeof(float);
 }
 
-cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& p, cudaStream_t st, int* launches) {
+size_t fast_fwd_workspace(const Problem& pb) {
+  return fast_fwd_supported(pb) ? (size_t)pb.units() * pb.T * kD * 2 : 0;
+}
+
+cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& p, void* keys_ws, cudaStream_t st,
+                            int* launches) {
   FastArgs a = {};
   a.B = pb.B; a.H = pb.H; a.T = pb.T; a.W = pb.W; a.n_off = pb.n_off; a.S = pb.S;
   a.n_tiles = (pb.T + kFastM - 1) / kFastM;
@@ -409,20 +497,44 @@ cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& p, cudaStream_t st
   std::sort(a.f, a.f + pb.n_off);
   const size_t smem = fast_fwd_smem(pb, &a.ring_rows, &a.sc_stride);
   a.q = reinterpret_cast<const __nv_bfloat16*>(p.q);
-  a.k = reinterpret_cast<const __nv_bfloat16*>(p.k);
   a.v = reinterpret_cast<const __nv_bfloat16*>(p.v);
   a.alpha = p.alpha; a.rope = p.rope;
   a.o = reinterpret_cast<__nv_bfloat16*>(p.o); a.lse = p.lse;
-  cudaError_t e = cudaFuncSetAttribute(k_fwd_fast, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&a.err), g_fwd_err);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((long long)pb.units() * a.n_tiles);
-  trace_mark("fwd_fast", st, true);
-  k_fwd_fast<<<grid, kFastM, smem, st>>>(a);
-  trace_mark("fwd_fast", st, false);
+  if (keys_ws) {
+    // rotated keys, fp16 of RoPE(K) / 256, then the staged kernel
+    if ((e = launch_rope_rows(p.k, p.rope, pb.T, pb.units() * pb.T, kKeyStage, keys_ws, st,
+                              "rope_keys")) != cudaSuccess)
+      return e;
+    a.k = keys_ws;
+    if ((e = cudaFuncSetAttribute(k_fwd_fast<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)) != cudaSuccess)
+      return e;
+    trace_mark("fwd_fast", st, true);
+    k_fwd_fast<true><<<grid, kFastM, smem, st>>>(a);
+    trace_mark("fwd_fast", st, false);
+    *launches += 1;
+  } else {
+    a.k = p.k;
+    if ((e = cudaFuncSetAttribute(k_fwd_fast<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)smem)) != cudaSuccess)
+      return e;
+    trace_mark("fwd_fast", st, true);
+    k_fwd_fast<false><<<grid, kFastM, smem, st>>>(a);
+    trace_mark("fwd_fast", st, false);
+  }
   e = cudaGetLastError();
   if (e == cudaSuccess) *launches += 1;
   return e;
+}
+
+cudaError_t fast_fwd_read_error(unsigned* out, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_fwd_err, sizeof(unsigned));
+  if (e != cudaSuccess || !clear || *out == 0) return e;
+  const unsigned zero = 0;
+  return cudaMemcpyToSymbol(g_fwd_err, &zero, sizeof(unsigned));
 }
 
 }  // namespace sa

@@ -54,10 +54,22 @@ void trace_mark(const char* kernel, cudaStream_t st, bool begin);
 
 // Each launcher returns the first CUDA error it saw and adds the number of
 // kernels it enqueued to *launches.
-// Staged bf16 / D=64 forward (sa_fast.cu).
+// Staged bf16 / D=64 forward (sa_fast.cu).  With keys_ws (fast_fwd_workspace
+// bytes) the keys are rotated once by the RoPE pre-pass; with nullptr raw K
+// rows are staged and rotated in shared memory (the allocation-free path).
 bool fast_fwd_supported(const Problem& pb);
 size_t fast_fwd_smem(const Problem& pb, int* ring_rows, int* sc_stride);
-cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& a, cudaStream_t st, int* launches);
+size_t fast_fwd_workspace(const Problem& pb);
+cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& a, void* keys_ws, cudaStream_t st,
+                            int* launches);
+// Device error words of the staged kernels (bit 0: a bounded staging wait
+// gave up); optionally cleared after reading.
+cudaError_t fast_fwd_read_error(unsigned* out, bool clear);
+
+// RoPE pre-pass (sa_prep.cu): y = fp16(RoPE(x) * mul) for n_rows rows of a bf16
+// [units][T][64] array, row r rotated at position r % T.
+cudaError_t launch_rope_rows(const void* x, const float2* rope, int T, long long n_rows, float mul,
+                             void* y, cudaStream_t st, const char* trace_name);
 
 // Staged bf16 / D=64 backward (sa_fast_bwd.cu).
 bool fast_bwd_supported(const Problem& pb);

@@ -69,9 +69,10 @@ def _p(**kw):
 
 def test_workspace_sizes(lib):
     f = lambda p, b: lib.sparse_attn_workspace_size(ctypes.byref(p), b)
-    assert f(_p(), 0) == 0
-    n = f(_p(), 1)
     units, T = 16 * 8 * 8, 1024
+    assert f(_p(), 0) == units * T * 64 * 2        # RoPE-rotated keys, 16-bit
+    assert f(_p(dtype=torch.float32), 0) == 0      # the general forward needs none
+    n = f(_p(), 1)
     assert n >= units * T * 4                      # D_i per query
     assert f(_p(sinks=4), 1) > n                   # sink partials
     assert f(_p(shape=(1, 1, 1, 1, 48)), 1) == 0   # unsupported D -> 0

@@ -175,7 +175,7 @@ def test_fast_path_is_the_one_dispatched():
         names = set(sa.trace_read())
     finally:
         sa.trace_enable(False)
-    assert names == {"fwd_fast"}, names
+    assert names == {"rope_keys", "fwd_fast"}, names
 
 
 @pytest.mark.parametrize("case", FAST, ids=[c[0] for c in FAST])
