@@ -34,6 +34,7 @@ FALLBACK_HBM_GBS = 6650.0
 #   forward  : read Q, K, V; write O and LSE
 #   bwd query: read Q, K, V, O, dO, LSE; write dQ and D
 #   bwd key  : read Q, K, V, dO, LSE, D; write dK, dV
+#   RoPE pre-pass (rope_keys / rope_queries): read K (or Q), write it rotated
 # (the whole backward: Q, K, V, O, dO, dQ, dK, dV and LSE = 1028 B)
 def alg_bytes_per_token_head(kernel, D, elt):
     row = D * elt
@@ -43,6 +44,8 @@ def alg_bytes_per_token_head(kernel, D, elt):
         return 6 * row + 8
     if kernel.startswith("bwd_kv"):
         return 6 * row + 8
+    if kernel.startswith("rope"):      # RoPE pre-pass: read a row, write it rotated
+        return 2 * row
     return 0
 
 

@@ -181,9 +181,11 @@ int32_t sparse_attn_trace_read(int32_t max, const char** names, double* total_ms
 }
 
 int32_t sparse_attn_device_error(int clear) {
-  unsigned fwd = 0;
-  if (sa::fast_fwd_read_error(&fwd, clear != 0) != cudaSuccess) return -1;
-  return (int32_t)fwd;
+  unsigned fwd = 0, bwd = 0;
+  if (sa::fast_fwd_read_error(&fwd, clear != 0) != cudaSuccess ||
+      sa::fast_bwd_read_error(&bwd, clear != 0) != cudaSuccess)
+    return -1;
+  return (int32_t)(fwd | bwd);
 }
 
 size_t sparse_attn_workspace_size(const sa_params* p, int backward) {

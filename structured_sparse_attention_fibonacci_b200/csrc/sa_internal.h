@@ -65,6 +65,7 @@ cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& a, void* keys_ws, 
 // Device error words of the staged kernels (bit 0: a bounded staging wait
 // gave up); optionally cleared after reading.
 cudaError_t fast_fwd_read_error(unsigned* out, bool clear);
+cudaError_t fast_bwd_read_error(unsigned* out, bool clear);
 
 // RoPE pre-pass (sa_prep.cu): y = fp16(RoPE(x) * mul) for n_rows rows of a bf16
 // [units][T][64] array, row r rotated at position r % T.

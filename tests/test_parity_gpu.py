@@ -209,4 +209,5 @@ def test_fast_backward_is_the_one_dispatched():
         names = set(sa.trace_read())
     finally:
         sa.trace_enable(False)
-    assert names == {"bwd_q_fast", "bwd_kv_fast", "reduce_dalpha"}, names
+    assert names == {"rope_keys", "rope_queries", "bwd_q_fast", "bwd_kv_fast",
+                     "reduce_dalpha"}, names
