@@ -179,6 +179,15 @@ int32_t sparse_attn_last_launch_count(void);
 void sparse_attn_force_general(int on);
 
 /*
+ * Diagnostics: which bf16 / D = 64 forward kernel sparse_attn_fwd runs.
+ * 0 (default): the faster for the configuration (tensor-core for windows of
+ * 32 or more, else CUDA-core); 1: the CUDA-core staged kernel; 2: the
+ * tensor-core kernel where it applies (at most 16 sinks).  Other values mean
+ * 0.  Process wide; sparse_attn_force_general takes precedence.
+ */
+void sparse_attn_select_forward(int which);
+
+/*
  * Kernel tracing (diagnostics).  While enabled (on != 0), every kernel the
  * library enqueues is bracketed by two CUDA events recorded on the same
  * stream.  sparse_attn_trace_read waits for all recorded events, writes up to

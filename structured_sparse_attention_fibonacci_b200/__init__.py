@@ -32,7 +32,7 @@ MAX_SINKS = 16
 EXPORTED = ("sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_workspace_size",
             "sparse_attn_status_string", "sparse_attn_last_launch_count",
             "sparse_attn_trace_enable", "sparse_attn_trace_read", "sparse_attn_force_general",
-            "sparse_attn_fwd_noalloc", "sparse_attn_device_error")
+            "sparse_attn_fwd_noalloc", "sparse_attn_device_error", "sparse_attn_select_forward")
 
 
 class SaParams(ctypes.Structure):
@@ -78,6 +78,8 @@ def lib():
         L.sparse_attn_last_launch_count.argtypes = []
         L.sparse_attn_force_general.restype = None
         L.sparse_attn_force_general.argtypes = [ctypes.c_int]
+        L.sparse_attn_select_forward.restype = None
+        L.sparse_attn_select_forward.argtypes = [ctypes.c_int]
         L.sparse_attn_device_error.restype = ctypes.c_int32
         L.sparse_attn_device_error.argtypes = [ctypes.c_int]
         L.sparse_attn_trace_enable.restype = None
@@ -128,6 +130,12 @@ def last_launch_count() -> int:
 def force_general(on: bool = True) -> None:
     """Route every call through the general kernels (diagnostics / testing)."""
     lib().sparse_attn_force_general(int(bool(on)))
+
+
+def select_forward(which: int = 0) -> None:
+    """Diagnostics: bf16 / d=64 forward kernel choice (0 auto, 1 CUDA-core
+    staged, 2 tensor-core); see sparse_attn_select_forward."""
+    lib().sparse_attn_select_forward(int(which))
 
 
 def device_error(clear: bool = True) -> int:

@@ -15,6 +15,7 @@ namespace {
 
 thread_local int32_t g_last_launches = 0;
 int g_force_general = 0;  // diagnostics: route every call through the general kernels
+int g_fwd_select = 0;     // diagnostics: 0 auto, 1 CUDA-core staged forward, 2 tensor-core forward
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -148,6 +149,8 @@ int32_t sparse_attn_last_launch_count(void) { return g_last_launches; }
 
 void sparse_attn_force_general(int on) { g_force_general = on != 0; }
 
+void sparse_attn_select_forward(int which) { g_fwd_select = (which == 1 || which == 2) ? which : 0; }
+
 void sparse_attn_trace_enable(int on) {
   std::lock_guard<std::mutex> lock(g_trace_mu);
   g_trace_on = on != 0;
@@ -181,11 +184,12 @@ int32_t sparse_attn_trace_read(int32_t max, const char** names, double* total_ms
 }
 
 int32_t sparse_attn_device_error(int clear) {
-  unsigned fwd = 0, bwd = 0;
+  unsigned fwd = 0, fwd_tc = 0, bwd = 0;
   if (sa::fast_fwd_read_error(&fwd, clear != 0) != cudaSuccess ||
+      sa::fast_fwd_tc_read_error(&fwd_tc, clear != 0) != cudaSuccess ||
       sa::fast_bwd_read_error(&bwd, clear != 0) != cudaSuccess)
     return -1;
-  return (int32_t)(fwd | bwd);
+  return (int32_t)(fwd | fwd_tc | bwd);
 }
 
 size_t sparse_attn_workspace_size(const sa_params* p, int backward) {
@@ -216,9 +220,14 @@ sa_status sparse_attn_fwd(const sa_params* p, const void* q, const void* k, cons
   if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
   sa::FwdPtrs a = {q, k, v, alpha, o, lse, rope};
   int launches = 0;
-  cudaError_t e = (!g_force_general && sa::fast_fwd_supported(pb))
-                      ? sa::launch_fwd_fast(pb, a, workspace, st, &launches)
-                      : sa::launch_fwd_general(pb, a, st, &launches);
+  cudaError_t e;
+  if (g_force_general || !sa::fast_fwd_supported(pb))
+    e = sa::launch_fwd_general(pb, a, st, &launches);
+  else if (g_fwd_select == 2 ? sa::tc_fwd_supported(pb)
+                              : (g_fwd_select == 0 && sa::tc_fwd_preferred(pb)))
+    e = sa::launch_fwd_tc(pb, a, workspace, st, &launches);
+  else
+    e = sa::launch_fwd_fast(pb, a, workspace, st, &launches);
   if (e != cudaSuccess) return SA_ERR_CUDA;
   g_last_launches = launches;
   return SA_OK;

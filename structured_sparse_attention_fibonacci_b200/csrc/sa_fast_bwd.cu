@@ -6,11 +6,14 @@
 // Query side (k_bwd_q_fast), one CTA per tile of 128 queries, three passes:
 //   1. K^ ring: scores sigma_m = q_hat . key_m and, per offset, the row-score
 //      difference dtau = q_hat . (K~[i-lo-1] - K~[i-lo]);
+//   owner lane: p_m = softmax of its own scores;
 //   2. V ring: dp_m = dO . value_m and dpi = dO . (V[i-lo-1] - V[i-lo]);
-//      owner lane: p_m = softmax of its own scores, D_i = sum_m p_m dp_m,
-//      g_m = p_m (dp_m - D_i), d-alpha += f_k (g_k dtau_k + p_k dpi_k)
-//      (the gradient through w_k = alpha f_k - lo_k: "Implementation" lets
-//      gradients reach alpha through the interpolation);
+//      owner lane: D_i = sum_m p_m dp_m, g_m = p_m (dp_m - D_i), and the
+//      d-alpha term sum_k f_k (g_k dtau_k + p_k dpi_k), the gradient through
+//      w_k = alpha f_k - lo_k ("Implementation" lets gradients reach alpha
+//      through the interpolation), accumulated as
+//        sum_k f_k p_k (dp_k dtau_k + dpi_k)  -  D_i sum_k f_k p_k dtau_k
+//      while pass 2 produces dp_k and dpi_k, so dpi is never stored;
 //   3. K^ ring again: dq_hat = sum_m g_m key_m, dQ = scale * RoPE^T(dq_hat).
 //   It also writes the weights the key side needs, indexed by KEY: for key j
 //   and lag d < W the folded window weight of query j + d (G for dK, P for
@@ -161,16 +164,19 @@ __device__ __forceinline__ void window_axpy(const unsigned char* ring, int RB, i
 
 // One pass of dot products of the lane's 4 rows `x` with every member
 // (window, sinks, far offsets) of the 16-bit array `src` (F16: rotated keys;
-// else V): member value into val_row, and for far offsets the row difference
-// (row b minus row a) into diff_row[k].  Returns nonzero when a staging wait
-// gave up.
+// else V): member value into val_row; for far offsets the row difference
+// (row b minus row a) goes to diff_row[k] (the key pass), or, with p_row set
+// (the value pass), into this query's d-alpha sum
+//   *dal_u += f_k p_k (dp_k dtau_k + dpi_k)      (diff_row then holds dtau).
+// Returns nonzero when a staging wait gave up.
 template <bool F16>
 __device__ __forceinline__ int member_dots(const FastBwdArgs& a, Stager& stg,
                                            unsigned char* ring, unsigned char* sinkb,
                                            const unsigned char* src, const OffGeo* sg,
                                            const int* s_kind, int i0, int ig, int c, int off0,
                                            int d1, const float (&x)[4][16], float* val_row,
-                                           float* diff_row, int i_own, float* mx) {
+                                           float* diff_row, int i_own, float* mx,
+                                           const float* p_row, float* dal_u) {
   constexpr int M = kFastM;
   const int T = a.T, W = a.W, S = a.S, RB = a.ring_rows;
   const int win_lo = i0 - W + 1, win_hi = i0 + M;
@@ -237,7 +243,12 @@ __device__ __forceinline__ int member_dots(const FastBwdArgs& a, Stager& stg,
       float out[2];
       reduce_scatter4<2>(part, out, c);
       val_row[W + S + kk] = out[0];
-      diff_row[kk] = out[1];
+      if (p_row) {
+        if (i_own - g.lo - 1 >= 0)
+          *dal_u += (float)g.f * p_row[W + S + kk] * (out[0] * diff_row[kk] + out[1]);
+      } else {
+        diff_row[kk] = out[1];
+      }
       if (mx && i_own - g.c >= 0) *mx = fmaxf(*mx, out[0]);
     }
     kb = nx;
@@ -258,7 +269,6 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
   float* sc = reinterpret_cast<float*>(sinkb + (size_t)S * kRowBytes);   // sigma, then g
   float* dpb = sc + (size_t)M * st;                                  // dp, then p
   float* dts = dpb + (size_t)M * st;                                 // [M][n_off] dtau
-  float* dps = dts + (size_t)M * n_off;                              // [M][n_off] dpi
   __shared__ OffGeo sg[SA_MAX_OFFSETS];
   __shared__ int s_kind[SA_MAX_OFFSETS];
   __shared__ float s_red[M / 32];
@@ -306,64 +316,79 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
   float* my_sc = sc + (size_t)lr * st;
   float* my_dp = dpb + (size_t)lr * st;
   float* my_dt = dts + (size_t)lr * n_off;
-  float* my_dpi = dps + (size_t)lr * n_off;
 
   float x[4][16];
   // pass 1: scores and row-score differences (rotated keys)
   load_lane_rows<true>(Q, a.rope, ig, T, c, par, a.scale * kKeyUnstage, x);
   float mx = -INFINITY;     // running max of this lane's query's valid scores
   if (member_dots<true>(a, stg, ring, sinkb, Kh, sg, s_kind, i0, ig, c, off0, d1, x, my_sc, my_dt,
-                        ig + c, &mx))
+                        ig + c, &mx, nullptr, nullptr))
     return;
-  // pass 2: dO . values and value differences
+
+  // owner lane: probabilities from these scores (not the forward's LSE, so
+  // that sum_m p_m = 1 and sum_m g_m = 0 hold for the values used here), and
+  // the first d-alpha sum  dal_v = sum_k f_k p_k dtau_k
+  const int i = ig + c;
+  const int n_slot = W + S + n_off;
+  float dal_v = 0.f, dal_u = 0.f;
+  if (i < T) {
+    for (int kk = 0; kk < n_off; ++kk) {
+      if (s_kind[kk] != kNear) continue;
+      const OffGeo g = sg[kk];
+      my_sc[W + S + kk] = g.wa * my_sc[g.lo] + g.w * my_sc[g.lo + 1];
+      my_dt[kk] = my_sc[g.lo + 1] - my_sc[g.lo];
+      if (i - g.c >= 0) mx = fmaxf(mx, my_sc[W + S + kk]);
+    }
+    float l = 0.f;
+    for (int m = 0; m < n_slot; ++m) {
+      bool valid;
+      if (m < W) valid = i - m >= 0;
+      else if (m < W + S) valid = m - W <= i;
+      else valid = s_kind[m - W - S] != kDead && i - sg[m - W - S].c >= 0;
+      const float e = valid ? __expf(my_sc[m] - mx) : 0.f;
+      my_sc[m] = e;
+      l += e;
+    }
+    const float inv = 1.f / l;
+    for (int m = 0; m < n_slot; ++m) my_sc[m] *= inv;          // scores -> p
+    for (int kk = 0; kk < n_off; ++kk) {
+      const OffGeo g = sg[kk];
+      if (s_kind[kk] != kDead && i - g.lo - 1 >= 0)
+        dal_v += (float)g.f * my_sc[W + S + kk] * my_dt[kk];
+    }
+  } else {
+    for (int m = 0; m < n_slot; ++m) my_sc[m] = 0.f;
+  }
+
+  // pass 2: dO . values; far offsets add f_k p_k (dp_k dtau_k + dpi_k) to dal_u
   load_lane_rows<false>(dO, a.rope, ig, T, c, par, 1.f, x);
   if (member_dots<false>(a, stg, ring, sinkb, Vb, sg, s_kind, i0, ig, c, off0, d1, x, my_dp,
-                         my_dpi, ig + c, nullptr))
+                         my_dt, ig + c, nullptr, my_sc, &dal_u))
     return;
   __syncthreads();
 
-  // owner lane: probabilities, D_i, dsigma, d-alpha, folded window weights
+  // owner lane: D_i, dsigma, d-alpha = dal_u - D_i dal_v, folded window weights
   float dal = 0.f;
   {
-    const int i = ig + c;
-    const int n_slot = W + S + n_off;
     if (i < T) {
-      for (int kk = 0; kk < n_off; ++kk) {
+      for (int kk = 0; kk < n_off; ++kk) {    // near offsets from two window values
         if (s_kind[kk] != kNear) continue;
         const OffGeo g = sg[kk];
-        my_sc[W + S + kk] = g.wa * my_sc[g.lo] + g.w * my_sc[g.lo + 1];
-        my_dp[W + S + kk] = g.wa * my_dp[g.lo] + g.w * my_dp[g.lo + 1];
-        my_dt[kk] = my_sc[g.lo + 1] - my_sc[g.lo];
-        my_dpi[kk] = my_dp[g.lo + 1] - my_dp[g.lo];
+        const float dpk = g.wa * my_dp[g.lo] + g.w * my_dp[g.lo + 1];
+        const float dpi = my_dp[g.lo + 1] - my_dp[g.lo];
+        my_dp[W + S + kk] = dpk;
+        if (i - g.lo - 1 >= 0)
+          dal_u += (float)g.f * my_sc[W + S + kk] * (dpk * my_dt[kk] + dpi);
       }
-      // softmax normalised from these scores (not the forward's LSE), so
-      // that sum_m p_m = 1 and sum_m g_m = 0 hold for the values used here
-      for (int kk = 0; kk < n_off; ++kk)      // near offsets join the running max
-        if (s_kind[kk] == kNear && i - sg[kk].c >= 0) mx = fmaxf(mx, my_sc[W + S + kk]);
-      float l = 0.f, edp = 0.f;
+      float Dsum = 0.f;
+      for (int m = 0; m < n_slot; ++m) Dsum += my_sc[m] != 0.f ? my_sc[m] * my_dp[m] : 0.f;
       for (int m = 0; m < n_slot; ++m) {
-        bool valid;
-        if (m < W) valid = i - m >= 0;
-        else if (m < W + S) valid = m - W <= i;
-        else valid = s_kind[m - W - S] != kDead && i - sg[m - W - S].c >= 0;
-        const float e = valid ? __expf(my_sc[m] - mx) : 0.f;
-        my_sc[m] = e;
-        l += e;
-        edp += valid ? e * my_dp[m] : 0.f;
-      }
-      const float inv = 1.f / l;
-      const float Dsum = edp * inv;
-      for (int m = 0; m < n_slot; ++m) {
-        const float p = my_sc[m] * inv;
+        const float p = my_sc[m];
         const float g = p * (my_dp[m] - Dsum);
         my_dp[m] = p;                       // dp -> p
-        my_sc[m] = p != 0.f ? g : 0.f;      // sc -> g (dsigma)
+        my_sc[m] = p != 0.f ? g : 0.f;      // p -> g (dsigma)
       }
-      for (int kk = 0; kk < n_off; ++kk) {
-        const OffGeo g = sg[kk];
-        if (s_kind[kk] != kDead && i - g.lo - 1 >= 0)
-          dal += (float)g.f * (my_sc[W + S + kk] * my_dt[kk] + my_dp[W + S + kk] * my_dpi[kk]);
-      }
+      dal = dal_u - Dsum * dal_v;
       for (int kk = 0; kk < n_off; ++kk) {  // fold near offsets into window weights
         if (s_kind[kk] != kNear) continue;
         const OffGeo g = sg[kk];
@@ -789,7 +814,7 @@ FastBwdLayout fast_bwd_layout(const Problem& pb) {
   const size_t ring_b = (size_t)(M / 32) * 2 * pb.S * kD * sizeof(float);
   const size_t ring_bytes = std::max(ring_a, ring_b);
   L.q_smem = ring_bytes + (size_t)pb.S * kRowBytes + 2 * (size_t)M * L.sc_stride * sizeof(float) +
-             2 * (size_t)M * pb.n_off * sizeof(float);
+             (size_t)M * pb.n_off * sizeof(float);
   L.kv_smem = ring_a + (size_t)L.NS * M * sizeof(__nv_bfloat16);
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   const size_t units = (size_t)pb.units();

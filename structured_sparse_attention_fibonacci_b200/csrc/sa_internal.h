@@ -62,6 +62,18 @@ size_t fast_fwd_smem(const Problem& pb, int* ring_rows, int* sc_stride);
 size_t fast_fwd_workspace(const Problem& pb);
 cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& a, void* keys_ws, cudaStream_t st,
                             int* launches);
+// Tensor-core bf16 / D=64 forward (sa_fwd_tc.cu); keys_ws as for the staged
+// forward (fast_fwd_workspace bytes, required).
+bool tc_fwd_supported(const Problem& pb);
+// Where the tensor-core forward is the faster one (long windows: measured on
+// B200, W = 64 runs 11% faster than the CUDA-core forward, W = 12 breaks even
+// on T = 1024 and is 8% slower on T = 4096).
+bool tc_fwd_preferred(const Problem& pb);
+size_t tc_fwd_smem(const Problem& pb, int* ring_rows, int* sc_stride);
+cudaError_t launch_fwd_tc(const Problem& pb, const FwdPtrs& a, void* keys_ws, cudaStream_t st,
+                          int* launches);
+cudaError_t fast_fwd_tc_read_error(unsigned* out, bool clear);
+
 // Device error words of the staged kernels (bit 0: a bounded staging wait
 // gave up); optionally cleared after reading.
 cudaError_t fast_fwd_read_error(unsigned* out, bool clear);

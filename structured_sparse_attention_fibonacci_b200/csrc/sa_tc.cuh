@@ -1,0 +1,125 @@
+// Tensor-core building blocks of the staged kernels: warp-level mma.sync
+// (m16n8k16 / m16n8k8, fp32 accumulate), ldmatrix fragment loads from a
+// 128-byte-swizzled row ring, and 3-D tensor-map (TMA) staging of 8-row boxes.
+//
+// Swizzled ring.  Row r of a 16-bit [T][64] array lives in slot
+// s = r & (RB - 1) (RB a power of two, >= 8) at byte s * 128, and its 16-byte
+// chunk c at position c ^ (s & 7): the layout the tensor copy writes with
+// 128-byte swizzling into a 1024-byte-aligned ring.  Eight consecutive rows
+// then put any one chunk in eight different bank groups, so an ldmatrix of
+// an 8 x 8 tile (eight rows, one chunk each) is conflict-free.  Boxes are 8
+// rows starting at a row that is a multiple of 8 (one 1024-byte swizzle atom
+// per box); rows outside [0, T) arrive zero-filled.
+//
+// The mma wrappers are plain (non-volatile) asm: pure register operations the
+// compiler may schedule; ldmatrix stays volatile (it reads shared memory) and
+// callers issue a tile's loads before its mma chain.
+//
+// Fragment layouts (PTX mma.m16n8k16, row-major A, column-major B), lane
+// l = 4 g + t:  A regs: (g, 2t..2t+1), (g+8, 2t..2t+1), (g, 2t+8..), (g+8, 2t+8..);
+// B regs: k = 2t..2t+1 and 2t+8..2t+9 of column g; C: (g, 2t), (g, 2t+1),
+// (g+8, 2t), (g+8, 2t+1).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "sa_stage.cuh"
+
+namespace sa {
+namespace tc {
+
+using stage::Stager;
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                        uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// m16n8k8: A regs (g, 2t..2t+1), (g+8, 2t..2t+1); B reg k = 2t..2t+1 of column g.
+__device__ __forceinline__ void mma_bf16_k8(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm(
+      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
+__device__ __forceinline__ void mma_f16_k8(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm(
+      "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Byte offset, within the ring, of 16-byte chunk `ch` of row `row`.
+__device__ __forceinline__ uint32_t swz_off(int row, int RB, int ch) {
+  const int slot = row & (RB - 1);
+  return (uint32_t)(slot * 128 + ((ch ^ (slot & 7)) << 4));
+}
+
+// One 8-row box of a 3-D [units][T][64] 16-bit tensor map (row coordinate may
+// be negative or >= T: zero fill) into shared memory at dst (1024-aligned).
+__device__ __forceinline__ void tma_rows8(uint32_t dst, const CUtensorMap* map, int row, int unit,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
+      "[%1, {%2, %3, %4}], [%5];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row), "r"(unit),
+      "r"(stage::smem_u32(bar))
+      : "memory");
+}
+
+// Register (thread 0) and issue the copies of rows [a, b) (multiples of 8,
+// b - a <= RB) of `unit` into the ring at ring_u32.  Completes on the round's
+// barrier (stage::stage_commit_wait).
+__device__ __forceinline__ void stage_tiles(Stager& s, uint32_t ring_u32, int RB,
+                                            const CUtensorMap* map, int unit, int a, int b) {
+  if (threadIdx.x != 0 || a >= b) return;
+  stage::mbar_expect_tx(s.bar, (uint32_t)(b - a) * 128u);
+  for (int r = a; r < b; r += 8)
+    tma_rows8(ring_u32 + (uint32_t)((r & (RB - 1)) * 128), map, r, unit, s.bar);
+}
+
+__device__ __forceinline__ int floor8(int x) { return x & ~7; }
+__device__ __forceinline__ int ceil8(int x) { return (x + 7) & ~7; }
+__device__ __forceinline__ int floor16(int x) { return x & ~15; }
+
+}  // namespace tc
+
+// Host: a 3-D tensor map over a 16-bit [units][T][64] array (boxes of 8 rows,
+// 128-byte swizzle, zero fill out of bounds).  sa_tmap.cu.
+cudaError_t make_rows_map(CUtensorMap* map, const void* base, int T, long long units);
+
+}  // namespace sa
