@@ -307,30 +307,69 @@ def run_ours(args, rank, world, local_rank):
         b = alg_bytes_per_token_head(n, wl.D, elt) * wl.token_heads
         kk["alg_GBps"] = b / (kk["ms_per_launch"] / 1e3) / 1e9 if b else None
 
-    # end to end through the public API: pinned host inputs in, results out
+    # End to end through the public API: every step copies its inputs in from
+    # pinned host memory and its results back out.  Two device buffer sets
+    # and three streams (copy in, compute, copy out) let step n's results
+    # travel to the host while step n+1's inputs arrive and step n+1 runs;
+    # a set is refilled only after its previous results have left.
     h_in = [t for t in host[:3]] + ([host[3]] if wl.backward else [])
-    d_in = [q, k, v] + ([do] if wl.backward else [])
-    outs = [o, lse] + ([dq, dk, dv, dal] if wl.backward else [])
-    h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
     h2d = sum(t.numel() * t.element_size() for t in h_in) + alpha_h.numel() * 4
-    d2h = sum(t.numel() * t.element_size() for t in outs)
+    sets = []
+    for b in range(2):
+        d_in = [torch.empty_like(t, device=dev) for t in h_in]
+        d_alpha = torch.empty_like(alpha)
+        d_out = [torch.empty_like(q), torch.empty(q.shape[:4], dtype=torch.float32, device=dev)]
+        if wl.backward:
+            d_out += [torch.empty_like(q), torch.empty_like(q), torch.empty_like(q),
+                      torch.empty(wl.L, dtype=torch.float32, device=dev)]
+        h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d_out]
+        sets.append((d_in, d_alpha, d_out, h_out))
+    d2h = sum(t.numel() * t.element_size() for t in sets[0][2])
+    s_in, s_run, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_run = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    started = [False, False]
 
-    def e2e_step():
-        for hs, ds in zip(h_in, d_in):
-            ds.copy_(hs, non_blocking=True)
-        alpha.copy_(alpha_h, non_blocking=True)
-        step()
-        for ho, do_ in zip(h_out, outs):
-            ho.copy_(do_, non_blocking=True)
+    def e2e_step(n):
+        b = n % 2
+        d_in, d_alpha, d_out, h_out = sets[b]
+        with torch.cuda.stream(s_in):
+            if started[b]:
+                s_in.wait_event(ev_out[b])        # this set's last results have left
+            for hs, ds in zip(h_in, d_in):
+                ds.copy_(hs, non_blocking=True)
+            d_alpha.copy_(alpha_h, non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(ev_in[b])
+            if wl.backward:
+                qq, kk_, vv, dd = d_in
+            else:
+                (qq, kk_, vv), dd = d_in, None
+            sa.fwd(qq, kk_, vv, d_alpha, out=d_out[0], lse=d_out[1], stream=s_run, **kw)
+            if wl.backward:
+                sa.bwd(qq, kk_, vv, d_out[0], d_out[1], dd, d_alpha, dq=d_out[2], dk=d_out[3],
+                       dv=d_out[4], dalpha=d_out[5], workspace=ws, stream=s_run, **kw)
+            ev_run[b].record(s_run)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_run[b])
+            for ho, dv_ in zip(h_out, d_out):
+                ho.copy_(dv_, non_blocking=True)
+            ev_out[b].record(s_out)
+        started[b] = True
 
-    e2e_step()
+    for n in range(2):
+        e2e_step(n)
     torch.cuda.synchronize()
     barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    f1.record(stream)
+    f0.record(s_in)
+    for n in range(args.steps):
+        e2e_step(n)
+    s_in.wait_stream(s_out)
+    s_in.wait_stream(s_run)
+    f1.record(s_in)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), dev)

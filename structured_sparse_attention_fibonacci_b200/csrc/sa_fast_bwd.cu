@@ -683,7 +683,7 @@ __device__ __forceinline__ int key_pass(const FastBwdArgs& a, Stager& stg, unsig
   return 0;
 }
 
-__global__ void __launch_bounds__(kFastM) k_bwd_kv_fast(const FastBwdArgs a) {
+__global__ void __launch_bounds__(kFastM, 4) k_bwd_kv_fast(const FastBwdArgs a) {
   constexpr int M = kFastM;
   extern __shared__ __align__(128) unsigned char smem[];
   const int T = a.T, S = a.S, RB = a.ring_rows, n_off = a.n_off;
