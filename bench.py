@@ -239,13 +239,18 @@ def run_ours(args, rank, world, local_rank):
         dal = torch.empty(wl.L, dtype=torch.float32, device=dev)
         ws = torch.empty(max(1, sa.workspace_size(tuple(q.shape), q.dtype, backward=True, **kw)),
                          dtype=torch.uint8, device=dev)
+        # training step: the forward saves what the backward reuses (rotated
+        # keys, probabilities, row-score differences) in a context buffer
+        n_ctx = sa.context_size(tuple(q.shape), q.dtype, **kw)
+        ctx = torch.empty(n_ctx, dtype=torch.uint8, device=dev) if n_ctx else None
     launches = [0]
 
     def step():
-        sa.fwd(q, k, v, alpha, out=o, lse=lse, **kw)
+        sa.fwd(q, k, v, alpha, out=o, lse=lse, context=ctx if wl.backward else None, **kw)
         n = sa.last_launch_count()
         if wl.backward:
-            sa.bwd(q, k, v, o, lse, do, alpha, dq=dq, dk=dk, dv=dv, dalpha=dal, workspace=ws, **kw)
+            sa.bwd(q, k, v, o, lse, do, alpha, dq=dq, dk=dk, dv=dv, dalpha=dal, workspace=ws,
+                   context=ctx, **kw)
             n += sa.last_launch_count()
         launches[0] += n
 
@@ -347,10 +352,12 @@ def run_ours(args, rank, world, local_rank):
                 qq, kk_, vv, dd = d_in
             else:
                 (qq, kk_, vv), dd = d_in, None
-            sa.fwd(qq, kk_, vv, d_alpha, out=d_out[0], lse=d_out[1], stream=s_run, **kw)
+            sa.fwd(qq, kk_, vv, d_alpha, out=d_out[0], lse=d_out[1], stream=s_run,
+                   context=ctx if wl.backward else None, **kw)
             if wl.backward:
                 sa.bwd(qq, kk_, vv, d_out[0], d_out[1], dd, d_alpha, dq=d_out[2], dk=d_out[3],
-                       dv=d_out[4], dalpha=d_out[5], workspace=ws, stream=s_run, **kw)
+                       dv=d_out[4], dalpha=d_out[5], workspace=ws, stream=s_run, context=ctx,
+                       **kw)
             ev_run[b].record(s_run)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_run[b])

@@ -131,6 +131,40 @@ sa_status sparse_attn_bwd(const sa_params* p, const void* q, const void* k, cons
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Training pair: a forward that also saves what the backward would otherwise
+ * recompute, and the backward that consumes it.  This is activation saving
+ * (the paper has no counterpart; its training runs a forward and a backward
+ * per step): the forward keeps, in the caller's `context` buffer,
+ *   - the RoPE-rotated keys (fp16 of RoPE(K) / 256, [L][B][H][T][D]),
+ *   - every member's softmax probability (window lags 0..W-1 unfolded, sinks,
+ *     offsets in the order of p->offsets sorted ascending), fp32
+ *     [L*B*H][W+S+n_offsets][T],
+ *   - every offset's row-score difference score(row i-lo-1) - score(row i-lo),
+ *     fp32 [L*B*H][n_offsets][T],
+ * and sparse_attn_bwd_ctx then skips the score pass and the key rotation.
+ * Results equal sparse_attn_fwd / sparse_attn_bwd up to fp32 rounding order.
+ *
+ * sparse_attn_context_size: bytes of the context for these params; 0 when
+ * the configuration has no staged kernels (dtype other than bf16 or D != 64):
+ * the two calls then return SA_ERR_UNSUPPORTED (use sparse_attn_fwd/_bwd).
+ * sparse_attn_fwd_train: arguments as sparse_attn_fwd, plus the context
+ * (device, >= sparse_attn_context_size bytes, 16-byte aligned; written).
+ * sparse_attn_bwd_ctx: arguments as sparse_attn_bwd plus the context written
+ * by sparse_attn_fwd_train for the same q, k, v, alpha and params (read; lse
+ * may be NULL); its workspace is sparse_attn_workspace_size(p, 1) bytes.
+ * Both run the staged kernels whatever sparse_attn_force_general says.
+ */
+size_t sparse_attn_context_size(const sa_params* p);
+sa_status sparse_attn_fwd_train(const sa_params* p, const void* q, const void* k, const void* v,
+                                const float* alpha, void* o, float* lse, void* context,
+                                size_t context_bytes, void* stream);
+sa_status sparse_attn_bwd_ctx(const sa_params* p, const void* q, const void* k, const void* v,
+                              const void* o, const float* lse, const void* dout,
+                              const float* alpha, const void* context, void* dq, void* dk,
+                              void* dv, float* dalpha, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
  * Forward that allocates no device memory.  The paper has no counterpart: this
  * entry point exists for callers that cannot let a library call cudaMalloc --
  * applications whose device memory belongs to a pooling allocator that must

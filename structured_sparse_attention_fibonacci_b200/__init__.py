@@ -32,7 +32,8 @@ MAX_SINKS = 16
 EXPORTED = ("sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_workspace_size",
             "sparse_attn_status_string", "sparse_attn_last_launch_count",
             "sparse_attn_trace_enable", "sparse_attn_trace_read", "sparse_attn_force_general",
-            "sparse_attn_fwd_noalloc", "sparse_attn_device_error", "sparse_attn_select_forward")
+            "sparse_attn_fwd_noalloc", "sparse_attn_device_error", "sparse_attn_select_forward",
+            "sparse_attn_context_size", "sparse_attn_fwd_train", "sparse_attn_bwd_ctx")
 
 
 class SaParams(ctypes.Structure):
@@ -78,6 +79,13 @@ def lib():
         L.sparse_attn_last_launch_count.argtypes = []
         L.sparse_attn_force_general.restype = None
         L.sparse_attn_force_general.argtypes = [ctypes.c_int]
+        L.sparse_attn_context_size.restype = ctypes.c_size_t
+        L.sparse_attn_context_size.argtypes = [P]
+        L.sparse_attn_fwd_train.restype = ctypes.c_int
+        L.sparse_attn_fwd_train.argtypes = [P, vp, vp, vp, fp, vp, fp, vp, ctypes.c_size_t, vp]
+        L.sparse_attn_bwd_ctx.restype = ctypes.c_int
+        L.sparse_attn_bwd_ctx.argtypes = [P, vp, vp, vp, vp, fp, vp, fp, vp, vp, vp, vp, fp, vp,
+                                          ctypes.c_size_t, vp]
         L.sparse_attn_select_forward.restype = None
         L.sparse_attn_select_forward.argtypes = [ctypes.c_int]
         L.sparse_attn_device_error.restype = ctypes.c_int32
@@ -181,13 +189,26 @@ def _check_tensors(shape, dtype, device, **named):
             raise ValueError(f"{name} must be {dtype} of shape {tuple(shape)}")
 
 
+def context_size(shape, dtype, **kw) -> int:
+    """Bytes of the training context (sparse_attn_context_size); 0 when the
+    configuration has no staged kernels."""
+    p = make_params(tuple(shape), dtype, **kw)
+    return int(lib().sparse_attn_context_size(ctypes.byref(p)))
+
+
 def fwd(q, k, v, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0, scale=0.0,
-        out=None, lse=None, want_lse=True, stream=None):
+        out=None, lse=None, want_lse=True, stream=None, context=None):
     """Sparse attention forward over all layers: returns (O, LSE or None).
 
     q, k, v: CUDA tensors [L, B, H, T, D] (bf16 or fp32, contiguous).
     alpha: CUDA fp32 [L].  Output buffers may be passed in via out= / lse=.
+    context: a CUDA uint8 buffer of context_size() bytes: the forward then
+    runs as sparse_attn_fwd_train and saves what bwd(..., context=) reuses.
     """
+    if context is not None:
+        return _fwd_train(q, k, v, alpha, window=window, offsets=offsets, sinks=sinks,
+                          rope_base=rope_base, scale=scale, out=out, lse=lse, want_lse=want_lse,
+                          stream=stream, context=context)
     shape, dtype, dev = tuple(q.shape), q.dtype, q.device
     if lse is None and want_lse:
         lse = torch.empty(shape[:4], dtype=torch.float32, device=dev)
@@ -201,6 +222,22 @@ def fwd(q, k, v, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0, sc
     st = L.sparse_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(out),
                            _ptr(lse), _ptr(ws), ws_n, _stream_handle(stream))
     _check("sparse_attn_fwd", st)
+    return out, lse
+
+
+def _fwd_train(q, k, v, alpha, *, window, offsets, sinks, rope_base, scale, out, lse, want_lse,
+               stream, context):
+    shape, dtype, dev = tuple(q.shape), q.dtype, q.device
+    if lse is None and want_lse:
+        lse = torch.empty(shape[:4], dtype=torch.float32, device=dev)
+    out = torch.empty_like(q) if out is None else out
+    _check_tensors(shape, dtype, dev, q=q, k=k, v=v, o=out, alpha=alpha, lse=lse)
+    p = make_params(shape, dtype, window=window, offsets=offsets, sinks=sinks,
+                    rope_base=rope_base, scale=scale)
+    st = lib().sparse_attn_fwd_train(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                     _ptr(out), _ptr(lse), _ptr(context), context.numel(),
+                                     _stream_handle(stream))
+    _check("sparse_attn_fwd_train", st)
     return out, lse
 
 
@@ -229,8 +266,12 @@ def fwd_noalloc(q, k, v, alpha, *, window, offsets=FIB15, sinks=0, rope_base=100
 
 
 def bwd(q, k, v, o, lse, dout, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0,
-        scale=0.0, dq=None, dk=None, dv=None, dalpha=None, workspace=None, stream=None):
-    """Sparse attention backward: returns (dQ, dK, dV, dalpha[L])."""
+        scale=0.0, dq=None, dk=None, dv=None, dalpha=None, workspace=None, stream=None,
+        context=None):
+    """Sparse attention backward: returns (dQ, dK, dV, dalpha[L]).
+
+    context: the buffer a fwd(..., context=) call filled for the same inputs;
+    the backward then runs as sparse_attn_bwd_ctx (no score pass)."""
     shape, dtype, dev = tuple(q.shape), q.dtype, q.device
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
@@ -244,6 +285,13 @@ def bwd(q, k, v, o, lse, dout, alpha, *, window, offsets=FIB15, sinks=0, rope_ba
     ws_n = int(L.sparse_attn_workspace_size(ctypes.byref(p), 1))
     if workspace is None or workspace.numel() < ws_n:
         workspace = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev)
+    if context is not None:
+        st = L.sparse_attn_bwd_ctx(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                   _ptr(dout), _ptr(alpha), _ptr(context), _ptr(dq), _ptr(dk),
+                                   _ptr(dv), _ptr(dalpha), _ptr(workspace), workspace.numel(),
+                                   _stream_handle(stream))
+        _check("sparse_attn_bwd_ctx", st)
+        return dq, dk, dv, dalpha
     st = L.sparse_attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                            _ptr(dout), _ptr(alpha), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dalpha),
                            _ptr(workspace), workspace.numel(), _stream_handle(stream))

@@ -233,6 +233,70 @@ sa_status sparse_attn_fwd(const sa_params* p, const void* q, const void* k, cons
   return SA_OK;
 }
 
+size_t sparse_attn_context_size(const sa_params* p) {
+  sa::Problem pb;
+  if (build_problem(p, &pb) != SA_OK) return 0;
+  if (!sa::fast_fwd_supported(pb) || !sa::fast_bwd_supported(pb)) return 0;
+  return sa::ctx_layout(pb).total;
+}
+
+sa_status sparse_attn_fwd_train(const sa_params* p, const void* q, const void* k, const void* v,
+                                const float* alpha, void* o, float* lse, void* context,
+                                size_t context_bytes, void* stream) {
+  sa::Problem pb;
+  sa_status s = build_problem(p, &pb);
+  if (s != SA_OK) return s;
+  if (!q || !k || !v || !alpha || !o) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse && !aligned4(lse)) || !aligned4(alpha))
+    return SA_ERR_INVALID_ARG;
+  const size_t need = sparse_attn_context_size(p);
+  if (need == 0) return SA_ERR_UNSUPPORTED;
+  if (context_bytes < need || !context || !aligned16(context)) return SA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float2* rope = nullptr;
+  if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
+  sa::FwdPtrs a = {q, k, v, alpha, o, lse, rope};
+  const sa::CtxLayout cl = sa::ctx_layout(pb);
+  char* cb = reinterpret_cast<char*>(context);
+  int launches = 0;
+  if (sa::launch_fwd_fast(pb, a, cb + cl.khat_off, st, &launches,
+                          reinterpret_cast<float*>(cb + cl.p_off),
+                          reinterpret_cast<float*>(cb + cl.dt_off)) != cudaSuccess)
+    return SA_ERR_CUDA;
+  g_last_launches = launches;
+  return SA_OK;
+}
+
+sa_status sparse_attn_bwd_ctx(const sa_params* p, const void* q, const void* k, const void* v,
+                              const void* o, const float* lse, const void* dout,
+                              const float* alpha, const void* context, void* dq, void* dk,
+                              void* dv, float* dalpha, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  sa::Problem pb;
+  sa_status s = build_problem(p, &pb);
+  if (s != SA_OK) return s;
+  const void* tensors[] = {q, k, v, o, dout, dq, dk, dv};
+  for (const void* x : tensors)
+    if (!x || !aligned16(x)) return SA_ERR_INVALID_ARG;
+  const void* vectors[] = {alpha, dalpha};
+  for (const void* x : vectors)
+    if (!x || !aligned4(x)) return SA_ERR_INVALID_ARG;
+  if (lse && !aligned4(lse)) return SA_ERR_INVALID_ARG;
+  if (sparse_attn_context_size(p) == 0) return SA_ERR_UNSUPPORTED;
+  if (!context || !aligned16(context)) return SA_ERR_INVALID_ARG;
+  const size_t need = sa::fast_bwd_workspace(pb);
+  if (workspace_bytes < need || !workspace || !aligned16(workspace)) return SA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float2* rope = nullptr;
+  if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
+  sa::BwdPtrs a = {q, k, v, o, dout, lse, alpha, dq, dk, dv, dalpha, rope, workspace};
+  int launches = 0;
+  if (sa::launch_bwd_fast(pb, a, st, &launches, context) != cudaSuccess) return SA_ERR_CUDA;
+  g_last_launches = launches;
+  return SA_OK;
+}
+
 sa_status sparse_attn_bwd(const sa_params* p, const void* q, const void* k, const void* v,
                           const void* o, const float* lse, const void* dout, const float* alpha,
                           void* dq, void* dk, void* dv, float* dalpha, void* workspace,

@@ -45,6 +45,8 @@ struct FastArgs {
   const float* alpha; const float2* rope;
   __nv_bfloat16* o; float* lse;
   unsigned* err;
+  float* save_p;                       // SAVE: [units][W+S+n_off][T] member probabilities
+  float* save_dt;                      // SAVE: [units][n_off][T] row-score differences
 };
 
 enum : int { kFar = 0, kNear = 1, kDead = 2 };
@@ -183,7 +185,13 @@ __device__ __forceinline__ int stage_keys(Stager& s, unsigned char* ring, int RB
   return 0;
 }
 
-template <bool PRE>
+// SAVE (training forward): also store, per query, every member's probability
+// (window lags unfolded, sinks, offsets) and every offset's row-score
+// difference dtau = score(row i-lo-1) - score(row i-lo), the values the
+// backward's score pass would recompute.  Offsets are then "near" only when
+// both rows lie in the window (lo + 1 <= W - 1), and far offsets always read
+// both rows.
+template <bool PRE, bool SAVE>
 __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
   constexpr int M = kFastM;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -212,7 +220,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
     const OffGeo g = offset_geometry(__ldg(a.alpha + layer), a.f[t]);
     sg[t] = g;
     bad = !g.ok;
-    const int near = g.ok && (g.lo + (g.w != 0.f ? 1 : 0) <= W - 1);
+    const int near = g.ok && (g.lo + ((SAVE || g.w != 0.f) ? 1 : 0) <= W - 1);
     const int dead = i0 + M - 1 - g.c < 0;        // no query of the tile has it yet
     s_kind[t] = near ? kNear : (dead ? kDead : kFar);
   }
@@ -314,7 +322,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
       }
       for (int m = kk; m < nx; m = next_far(s_kind, m, n_off)) {
         const OffGeo g = sg[m];
-        const int two = g.w != 0.f;
+        const int two = SAVE || g.w != 0.f;
         const unsigned char* p = ring + (size_t)((ig - g.lo - 1) & (RB - 1)) * kRowBytes + off0;
         float pa[4] = {0.f, 0.f, 0.f, 0.f}, pb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -325,12 +333,17 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
           if (u <= 3) pb[u] = dot16(q[u], x);
           if (u >= 1) pa[u - 1] = dot16(q[u - 1], x);
         }
-        float part[4][1];
+        constexpr int NV = SAVE ? 2 : 1;
+        float part[4][NV];
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) part[qq][0] = g.wa * pa[qq] + g.w * pb[qq];
-        float out[1];
-        reduce_scatter4<1>(part, out, c);
+        for (int qq = 0; qq < 4; ++qq) {
+          part[qq][0] = g.wa * pa[qq] + g.w * pb[qq];
+          if (SAVE) part[qq][NV - 1] = pb[qq] - pa[qq];
+        }
+        float out[NV];
+        reduce_scatter4<NV>(part, out, c);
         my_sc[W + S + m] = out[0];
+        if (SAVE && i_own < T) a.save_dt[((size_t)unit * n_off + m) * T + i_own] = out[NV - 1];
         if (i_own - g.c >= 0) mx = fmaxf(mx, out[0]);
       }
       kk = nx;
@@ -346,11 +359,14 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
     const int i = i_own;
     if (i < T) {
       for (int kk = 0; kk < n_off; ++kk) {    // near offsets: from two window scores
+        if (SAVE && s_kind[kk] == kDead) a.save_dt[((size_t)unit * n_off + kk) * T + i] = 0.f;
         if (s_kind[kk] != kNear) continue;
         const OffGeo g = sg[kk];
         float sv = g.wa * my_sc[g.lo];
         if (g.w != 0.f) sv += g.w * my_sc[g.lo + 1];
         my_sc[W + S + kk] = sv;
+        if (SAVE)
+          a.save_dt[((size_t)unit * n_off + kk) * T + i] = my_sc[g.lo + 1] - my_sc[g.lo];
         if (i - g.c >= 0) mx = fmaxf(mx, sv);
       }
       float l = 0.f;
@@ -364,14 +380,22 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
       }
       for (int kk = 0; kk < n_off; ++kk) {
         const OffGeo g = sg[kk];
-        const float e = (i - g.c >= 0) ? __expf(my_sc[W + S + kk] - mx) : 0.f;
+        const float e =
+            (s_kind[kk] != kDead && i - g.c >= 0) ? __expf(my_sc[W + S + kk] - mx) : 0.f;
         my_sc[W + S + kk] = e; l += e;
-        if (s_kind[kk] == kNear) {             // fold into the two window weights
-          my_sc[g.lo] += g.wa * e;
-          if (g.w != 0.f) my_sc[g.lo + 1] += g.w * e;
-        }
       }
       inv_l = 1.f / l;
+      if (SAVE) {                              // probabilities, window lags unfolded
+        float* sp = a.save_p + (size_t)unit * (W + S + n_off) * T + i;
+        for (int m = 0; m < W + S + n_off; ++m) sp[(size_t)m * T] = my_sc[m] * inv_l;
+      }
+      for (int kk = 0; kk < n_off; ++kk) {     // fold near offsets into the window weights
+        if (s_kind[kk] != kNear) continue;
+        const OffGeo g = sg[kk];
+        const float e = my_sc[W + S + kk];
+        my_sc[g.lo] += g.wa * e;
+        if (g.w != 0.f) my_sc[g.lo + 1] += g.w * e;
+      }
       if (a.lse) a.lse[(size_t)unit * T + i] = mx + __logf(l);
     } else {
       for (int d = 0; d < W + S + n_off; ++d) my_sc[d] = 0.f;
@@ -488,7 +512,7 @@ size_t fast_fwd_workspace(const Problem& pb) {
 }
 
 cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& p, void* keys_ws, cudaStream_t st,
-                            int* launches) {
+                            int* launches, float* save_p, float* save_dt) {
   FastArgs a = {};
   a.B = pb.B; a.H = pb.H; a.T = pb.T; a.W = pb.W; a.n_off = pb.n_off; a.S = pb.S;
   a.n_tiles = (pb.T + kFastM - 1) / kFastM;
@@ -500,32 +524,31 @@ cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& p, void* keys_ws, 
   a.v = reinterpret_cast<const __nv_bfloat16*>(p.v);
   a.alpha = p.alpha; a.rope = p.rope;
   a.o = reinterpret_cast<__nv_bfloat16*>(p.o); a.lse = p.lse;
+  a.save_p = save_p; a.save_dt = save_dt;
   cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&a.err), g_fwd_err);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((long long)pb.units() * a.n_tiles);
+  auto launch = [&](auto kernel) -> cudaError_t {
+    cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (r != cudaSuccess) return r;
+    trace_mark("fwd_fast", st, true);
+    kernel<<<grid, kFastM, smem, st>>>(a);
+    trace_mark("fwd_fast", st, false);
+    return cudaGetLastError();
+  };
   if (keys_ws) {
     // rotated keys, fp16 of RoPE(K) / 256, then the staged kernel
     if ((e = launch_rope_rows(p.k, p.rope, pb.T, pb.units() * pb.T, kKeyStage, keys_ws, st,
                               "rope_keys")) != cudaSuccess)
       return e;
-    a.k = keys_ws;
-    if ((e = cudaFuncSetAttribute(k_fwd_fast<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)smem)) != cudaSuccess)
-      return e;
-    trace_mark("fwd_fast", st, true);
-    k_fwd_fast<true><<<grid, kFastM, smem, st>>>(a);
-    trace_mark("fwd_fast", st, false);
     *launches += 1;
+    a.k = keys_ws;
+    e = (save_p && save_dt) ? launch(k_fwd_fast<true, true>) : launch(k_fwd_fast<true, false>);
   } else {
     a.k = p.k;
-    if ((e = cudaFuncSetAttribute(k_fwd_fast<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)smem)) != cudaSuccess)
-      return e;
-    trace_mark("fwd_fast", st, true);
-    k_fwd_fast<false><<<grid, kFastM, smem, st>>>(a);
-    trace_mark("fwd_fast", st, false);
+    e = launch(k_fwd_fast<false, false>);
   }
-  e = cudaGetLastError();
   if (e == cudaSuccess) *launches += 1;
   return e;
 }

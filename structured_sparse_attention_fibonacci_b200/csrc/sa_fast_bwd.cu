@@ -52,6 +52,8 @@ struct FastBwdArgs {
   float* dal_part;                       // [units][n_tiles]
   float* sink_k; float* sink_v;          // [units][n_tiles][S][64]
   unsigned* err;
+  const float* ctx_p;                    // training context: [units][W+S+n_off][T] probabilities
+  const float* ctx_dt;                   // ... and [units][n_off][T] row-score differences
 };
 
 enum : int { kFar = 0, kNear = 1, kDead = 2 };
@@ -256,6 +258,9 @@ __device__ __forceinline__ int member_dots(const FastBwdArgs& a, Stager& stg,
   return 0;
 }
 
+// CTX: the probabilities and row-score differences come from the training
+// context the saving forward wrote; the score pass is skipped.
+template <bool CTX>
 __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
   constexpr int M = kFastM;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -318,46 +323,59 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
   float* my_dt = dts + (size_t)lr * n_off;
 
   float x[4][16];
-  // pass 1: scores and row-score differences (rotated keys)
-  load_lane_rows<true>(Q, a.rope, ig, T, c, par, a.scale * kKeyUnstage, x);
-  float mx = -INFINITY;     // running max of this lane's query's valid scores
-  if (member_dots<true>(a, stg, ring, sinkb, Kh, sg, s_kind, i0, ig, c, off0, d1, x, my_sc, my_dt,
-                        ig + c, &mx, nullptr, nullptr))
-    return;
-
-  // owner lane: probabilities from these scores (not the forward's LSE, so
-  // that sum_m p_m = 1 and sum_m g_m = 0 hold for the values used here), and
-  // the first d-alpha sum  dal_v = sum_k f_k p_k dtau_k
   const int i = ig + c;
   const int n_slot = W + S + n_off;
   float dal_v = 0.f, dal_u = 0.f;
+  if (CTX) {
+    // probabilities and row-score differences from the training context
+    if (i < T) {
+      const float* cp = a.ctx_p + (size_t)unit * n_slot * T + i;
+      const float* cd = a.ctx_dt + (size_t)unit * n_off * T + i;
+      for (int m = 0; m < n_slot; ++m) my_sc[m] = __ldg(cp + (size_t)m * T);
+      for (int kk = 0; kk < n_off; ++kk) my_dt[kk] = __ldg(cd + (size_t)kk * T);
+    } else {
+      for (int m = 0; m < n_slot; ++m) my_sc[m] = 0.f;
+    }
+  } else {
+    // pass 1: scores and row-score differences (rotated keys)
+    load_lane_rows<true>(Q, a.rope, ig, T, c, par, a.scale * kKeyUnstage, x);
+    float mx = -INFINITY;   // running max of this lane's query's valid scores
+    if (member_dots<true>(a, stg, ring, sinkb, Kh, sg, s_kind, i0, ig, c, off0, d1, x, my_sc,
+                          my_dt, ig + c, &mx, nullptr, nullptr))
+      return;
+    // owner lane: probabilities from these scores (not the forward's LSE, so
+    // that sum_m p_m = 1 and sum_m g_m = 0 hold for the values used here)
+    if (i < T) {
+      for (int kk = 0; kk < n_off; ++kk) {
+        if (s_kind[kk] != kNear) continue;
+        const OffGeo g = sg[kk];
+        my_sc[W + S + kk] = g.wa * my_sc[g.lo] + g.w * my_sc[g.lo + 1];
+        my_dt[kk] = my_sc[g.lo + 1] - my_sc[g.lo];
+        if (i - g.c >= 0) mx = fmaxf(mx, my_sc[W + S + kk]);
+      }
+      float l = 0.f;
+      for (int m = 0; m < n_slot; ++m) {
+        bool valid;
+        if (m < W) valid = i - m >= 0;
+        else if (m < W + S) valid = m - W <= i;
+        else valid = s_kind[m - W - S] != kDead && i - sg[m - W - S].c >= 0;
+        const float e = valid ? __expf(my_sc[m] - mx) : 0.f;
+        my_sc[m] = e;
+        l += e;
+      }
+      const float inv = 1.f / l;
+      for (int m = 0; m < n_slot; ++m) my_sc[m] *= inv;          // scores -> p
+    } else {
+      for (int m = 0; m < n_slot; ++m) my_sc[m] = 0.f;
+    }
+  }
+  // the first d-alpha sum  dal_v = sum_k f_k p_k dtau_k
   if (i < T) {
-    for (int kk = 0; kk < n_off; ++kk) {
-      if (s_kind[kk] != kNear) continue;
-      const OffGeo g = sg[kk];
-      my_sc[W + S + kk] = g.wa * my_sc[g.lo] + g.w * my_sc[g.lo + 1];
-      my_dt[kk] = my_sc[g.lo + 1] - my_sc[g.lo];
-      if (i - g.c >= 0) mx = fmaxf(mx, my_sc[W + S + kk]);
-    }
-    float l = 0.f;
-    for (int m = 0; m < n_slot; ++m) {
-      bool valid;
-      if (m < W) valid = i - m >= 0;
-      else if (m < W + S) valid = m - W <= i;
-      else valid = s_kind[m - W - S] != kDead && i - sg[m - W - S].c >= 0;
-      const float e = valid ? __expf(my_sc[m] - mx) : 0.f;
-      my_sc[m] = e;
-      l += e;
-    }
-    const float inv = 1.f / l;
-    for (int m = 0; m < n_slot; ++m) my_sc[m] *= inv;          // scores -> p
     for (int kk = 0; kk < n_off; ++kk) {
       const OffGeo g = sg[kk];
       if (s_kind[kk] != kDead && i - g.lo - 1 >= 0)
         dal_v += (float)g.f * my_sc[W + S + kk] * my_dt[kk];
     }
-  } else {
-    for (int m = 0; m < n_slot; ++m) my_sc[m] = 0.f;
   }
 
   // pass 2: dO . values; far offsets add f_k p_k (dp_k dtau_k + dpi_k) to dal_u
@@ -847,7 +865,8 @@ cudaError_t fast_bwd_read_error(unsigned* out, bool clear) {
   return cudaMemcpyToSymbol(g_bwd_err, &zero, sizeof(unsigned));
 }
 
-cudaError_t launch_bwd_fast(const Problem& pb, const BwdPtrs& p, cudaStream_t st, int* launches) {
+cudaError_t launch_bwd_fast(const Problem& pb, const BwdPtrs& p, cudaStream_t st, int* launches,
+                            const void* ctx) {
   const FastBwdLayout L = fast_bwd_layout(pb);
   FastBwdArgs a = {};
   a.B = pb.B; a.H = pb.H; a.T = pb.T; a.W = pb.W; a.n_off = pb.n_off; a.S = pb.S;
@@ -864,8 +883,14 @@ cudaError_t launch_bwd_fast(const Problem& pb, const BwdPtrs& p, cudaStream_t st
   a.dk = reinterpret_cast<__nv_bfloat16*>(p.dk);
   a.dv = reinterpret_cast<__nv_bfloat16*>(p.dv);
   char* ws = reinterpret_cast<char*>(p.workspace);
-  void* khat = ws + L.khat_off;
+  const CtxLayout CL = ctx_layout(pb);
+  const char* cb = reinterpret_cast<const char*>(ctx);
+  void* khat = ctx ? const_cast<char*>(cb + CL.khat_off) : ws + L.khat_off;
   void* qhat = ws + L.qhat_off;
+  if (ctx) {
+    a.ctx_p = reinterpret_cast<const float*>(cb + CL.p_off);
+    a.ctx_dt = reinterpret_cast<const float*>(cb + CL.dt_off);
+  }
   a.khat = khat;
   a.qhat = qhat;
   a.gblk = reinterpret_cast<__nv_bfloat16*>(ws + L.gblk_off);
@@ -877,13 +902,14 @@ cudaError_t launch_bwd_fast(const Problem& pb, const BwdPtrs& p, cudaStream_t st
   if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&a.err), g_bwd_err)) != cudaSuccess)
     return e;
   const long long n_rows = pb.units() * pb.T;
-  if ((e = launch_rope_rows(p.k, p.rope, pb.T, n_rows, kKeyStage, khat, st, "rope_keys")) !=
-      cudaSuccess)
+  if (!ctx && (e = launch_rope_rows(p.k, p.rope, pb.T, n_rows, kKeyStage, khat, st,
+                                    "rope_keys")) != cudaSuccess)
     return e;
   if ((e = launch_rope_rows(p.q, p.rope, pb.T, n_rows, pb.scale * kKeyStage, qhat, st,
                             "rope_queries")) != cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(k_bwd_q_fast, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kq = ctx ? k_bwd_q_fast<true> : k_bwd_q_fast<false>;
+  if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)L.q_smem)) != cudaSuccess)
     return e;
   if ((e = cudaFuncSetAttribute(k_bwd_kv_fast, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -891,7 +917,7 @@ cudaError_t launch_bwd_fast(const Problem& pb, const BwdPtrs& p, cudaStream_t st
     return e;
   const unsigned grid = (unsigned)((long long)pb.units() * L.n_tiles);
   trace_mark("bwd_q_fast", st, true);
-  k_bwd_q_fast<<<grid, kFastM, L.q_smem, st>>>(a);
+  kq<<<grid, kFastM, L.q_smem, st>>>(a);
   trace_mark("bwd_q_fast", st, false);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   trace_mark("bwd_kv_fast", st, true);
@@ -901,7 +927,7 @@ cudaError_t launch_bwd_fast(const Problem& pb, const BwdPtrs& p, cudaStream_t st
   if ((e = launch_reduce_dalpha(a.dal_part, pb.L, pb.B * pb.H * L.n_tiles, p.dalpha, st)) !=
       cudaSuccess)
     return e;
-  *launches += 5;
+  *launches += ctx ? 4 : 5;
   return cudaSuccess;
 }
 

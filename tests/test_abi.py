@@ -116,3 +116,27 @@ def test_python_binding_refuses_cpu_tensors(lib):
     q = torch.zeros((1, 1, 1, 8, 16))
     with pytest.raises((ValueError, RuntimeError)):
         sa.fwd(q, q, q, torch.ones(1), window=2)
+
+
+def test_context_size_and_validation(lib):
+    """The training context exists only for the staged configurations, and
+    the training calls reject a missing or short context before any GPU work."""
+    f = lambda p: lib.sparse_attn_context_size(ctypes.byref(p))
+    units, T = 16 * 8 * 8, 1024
+    n = f(_p())
+    assert n >= units * T * (64 * 2 + 4 * (12 + 15 + 15))
+    assert f(_p(dtype=torch.float32)) == 0
+    assert f(_p(shape=(1, 1, 1, 64, 32))) == 0
+    dummy = ctypes.c_void_p(1 << 20)     # never dereferenced: validation comes first
+    p32 = _p(dtype=torch.float32, shape=(1, 1, 1, 64, 64))
+    alpha = ctypes.c_void_p(1 << 20)
+    st = lib.sparse_attn_fwd_train(ctypes.byref(p32), dummy, dummy, dummy, alpha, dummy, None,
+                                   dummy, 1 << 30, None)
+    assert st == sa.SA_ERR_UNSUPPORTED
+    p16 = _p(shape=(1, 1, 1, 64, 64))
+    st = lib.sparse_attn_fwd_train(ctypes.byref(p16), dummy, dummy, dummy, alpha, dummy, None,
+                                   dummy, 16, None)
+    assert st == sa.SA_ERR_WORKSPACE
+    st = lib.sparse_attn_bwd_ctx(ctypes.byref(p16), dummy, dummy, dummy, dummy, None, dummy,
+                                 alpha, None, dummy, dummy, dummy, alpha, dummy, 1 << 30, None)
+    assert st == sa.SA_ERR_INVALID_ARG

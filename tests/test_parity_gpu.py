@@ -217,6 +217,46 @@ def test_fast_and_general_backward(case):
     check_bwd(g_gen, ref, torch.bfloat16, name + " (general)")
 
 
+@pytest.mark.parametrize("case", FAST, ids=[c[0] for c in FAST])
+def test_training_context_forward_and_backward(case):
+    """sparse_attn_fwd_train + sparse_attn_bwd_ctx against the oracle (the
+    backward reuses the forward's probabilities, row-score differences and
+    rotated keys instead of recomputing them)."""
+    name, shape, W, S, alphas, offs = case
+    q, k, v, do = _inputs(shape, torch.bfloat16, seed=zlib.crc32(name.encode()) % 10000 + 1)
+    alpha = torch.tensor(alphas, dtype=torch.float32, device=DEV)
+    kw = dict(window=W, sinks=S, offsets=offs)
+    n_ctx = sa.context_size(shape, torch.bfloat16, **kw)
+    assert n_ctx > 0
+    ctx = torch.full((n_ctx,), 0xFF, dtype=torch.uint8, device=DEV)   # NaN-filled on purpose
+    o, lse = sa.fwd(q, k, v, alpha, context=ctx, **kw)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle_fwd(q, k, v, alpha, **kw)
+    check_fwd(o, lse, o_ref, lse_ref, torch.bfloat16, name + " (training forward)")
+    g = sa.bwd(q, k, v, o, None, do, alpha, context=ctx, **kw)
+    torch.cuda.synchronize()
+    ref = oracle_bwd(q, k, v, do, alpha, **kw)
+    check_bwd(g, ref, torch.bfloat16, name + " (context backward)")
+
+
+def test_training_context_dispatch_skips_the_score_pass():
+    q, k, v, do = _inputs((1, 1, 1, 300, 64), torch.bfloat16, seed=7)
+    alpha = torch.tensor([1.1], device=DEV)
+    ctx = torch.empty(sa.context_size(tuple(q.shape), q.dtype, window=12), dtype=torch.uint8,
+                      device=DEV)
+    sa.trace_enable(True)
+    try:
+        o, lse = sa.fwd(q, k, v, alpha, window=12, context=ctx)
+        sa.bwd(q, k, v, o, lse, do, alpha, window=12, context=ctx)
+        names = set(sa.trace_read())
+    finally:
+        sa.trace_enable(False)
+    # one key rotation (the forward's), no second one in the backward
+    assert names == {"rope_keys", "fwd_fast", "rope_queries", "bwd_q_fast", "bwd_kv_fast",
+                     "reduce_dalpha"}, names
+    assert sa.device_error() == 0
+
+
 def test_fast_backward_is_the_one_dispatched():
     q, k, v, do = _inputs((1, 1, 1, 300, 64), torch.bfloat16, seed=6)
     alpha = torch.tensor([1.0], device=DEV)
