@@ -327,12 +327,14 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
   const int n_slot = W + S + n_off;
   float dal_v = 0.f, dal_u = 0.f;
   if (CTX) {
-    // probabilities and row-score differences from the training context
+    // probabilities and row-score differences from the training context:
+    // every element an asynchronous 4-byte copy into this lane's rows, one wait
     if (i < T) {
       const float* cp = a.ctx_p + (size_t)unit * n_slot * T + i;
       const float* cd = a.ctx_dt + (size_t)unit * n_off * T + i;
-      for (int m = 0; m < n_slot; ++m) my_sc[m] = __ldg(cp + (size_t)m * T);
-      for (int kk = 0; kk < n_off; ++kk) my_dt[kk] = __ldg(cd + (size_t)kk * T);
+      for (int m = 0; m < n_slot; ++m) cp_async4(my_sc + m, cp + (size_t)m * T);
+      for (int kk = 0; kk < n_off; ++kk) cp_async4(my_dt + kk, cd + (size_t)kk * T);
+      cp_async_wait_all();
     } else {
       for (int m = 0; m < n_slot; ++m) my_sc[m] = 0.f;
     }
@@ -446,19 +448,20 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
       for (int m = 0; m < n_slot; ++m) { my_sc[m] = 0.f; my_dp[m] = 0.f; }
     }
     // zero the weight entries of this tile's keys that no query writes
-    // (source query at or beyond T; near-offset slots are never read)
+    // (source query at or beyond T; near-offset slots are never read): per
+    // slot the keys [max(i0, T - lag), min(i0 + M, T)), one warp per slot
     {
       const size_t base = ((size_t)unit * a.n_tiles + tile) * (size_t)a.NS * M;
-      for (int e = t; e < a.NS * M; e += M) {
-        const int slot = e / M, j = i0 + e % M;
-        if (j >= T) continue;
+      const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
+      for (int slot = warp; slot < a.NS; slot += M / 32) {
         int lag;
         if (slot < W) lag = slot;
         else if (slot < W + n_off) lag = sg[slot - W].lo;
         else lag = sg[slot - W - n_off].lo + 1;
-        if (j + lag >= T) {
-          a.gblk[base + e] = __float2bfloat16_rn(0.f);
-          a.pblk[base + e] = __float2bfloat16_rn(0.f);
+        const int jhi = min(i0 + M, T);
+        for (int j = max(i0, T - lag) + lane; j < jhi; j += 32) {
+          a.gblk[base + (size_t)slot * M + (j - i0)] = zero;
+          a.pblk[base + (size_t)slot * M + (j - i0)] = zero;
         }
       }
     }

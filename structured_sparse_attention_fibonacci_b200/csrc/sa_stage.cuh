@@ -187,6 +187,15 @@ __device__ __forceinline__ void stage_plain(Stager& s, unsigned char* buf, const
   bulk_copy(buf, src, (uint32_t)n_valid * kRowBytes, s.bar);
 }
 
+// Asynchronous 4-byte global -> shared copy (completes at cp_async_wait_all).
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
+}
+
 // ---- lane access ------------------------------------------------------------
 // Byte offsets, within a row, of the two 16-byte chunks lane (group parity
 // `par`, lane-in-group c) holds: first half, second half.
