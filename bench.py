@@ -52,7 +52,11 @@ def alg_bytes_per_token_head(kernel, D, elt):
 # dram__bytes_read.sum + dram__bytes_write.sum per token-head from the ncu
 # captures summarised under profiles/, keyed by kernel and the hash of the
 # kernel sources they were taken on; a changed source reports null.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    # profiles/staged_kernels_learned_train.md: 579.8 + 238.6 MB per launch of
+    # the context-mode query side over 1048576 token-heads
+    "bwd_q_fast@20d57b6d526b": 780.5,
+}
 
 
 def kernel_source_hash():
