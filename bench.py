@@ -49,6 +49,14 @@ def alg_bytes_per_token_head(kernel, D, elt):
     return 0
 
 
+def decode_bytes_per_token_head(wl, elt):
+    """Decode: read the query and every K and V row of its attended set (W
+    window rows, the sinks, two rows per offset); write O and LSE."""
+    row = wl.D * elt
+    rows = wl.window + wl.sinks + 2 * len(wl.offsets)
+    return 2 * row + 4 + 2 * rows * row
+
+
 # dram__bytes_read.sum + dram__bytes_write.sum per token-head from the ncu
 # captures summarised under profiles/, keyed by kernel and the hash of the
 # kernel sources they were taken on; a changed source reports null.
@@ -165,6 +173,21 @@ def oracle_sample(wl, budget_s):
               precision="f32")
     alpha = wl.alpha().numpy()
 
+    if wl.decode:
+        from structured_sparse_attention_fibonacci_b200.inputs import make_decode_inputs
+        q1, kc, vc = (t.float().numpy() for t in make_decode_inputs(wl))
+        reps, t = 0, 0.0
+        while reps == 0 or (t < budget_s and reps < 1000):
+            t0 = time.perf_counter()
+            oracle.decode(q1, kc, vc, alpha, wl.T - 1, **kw)
+            t += time.perf_counter() - t0
+            reps += 1
+        cores = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+        units = wl.L * wl.B * wl.H
+        return {"value": reps * units / t, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"{reps} decode steps of {units} (layer, batch, head) units at "
+                          f"position {wl.T - 1}, fp32 oracle", "seconds": round(t, 3)}
+
     def one_layer(l):
         ts = make_inputs(wl, layers=range(l, l + 1))
         arr = [t.float().numpy() for t in ts]
@@ -213,11 +236,16 @@ def run_reference(args, rank, world):
 
 
 def workload_config(wl, world):
+    if wl.decode:
+        pass_ = f"decode (one token at position {wl.T - 1}, KV cache of {wl.T} rows)"
+    else:
+        pass_ = "forward+backward" if wl.backward else "forward"
     return {"workload": wl.name, "L": wl.L, "B": wl.B, "H": wl.H, "T": wl.T, "D": wl.D,
             "window": wl.window, "sinks": wl.sinks, "offsets": "fib15 (1..987)",
-            "alpha": wl.alpha_kind, "pass": "forward+backward" if wl.backward else "forward",
+            "alpha": wl.alpha_kind, "pass": pass_,
             "global_batch": wl.B * world, "seq_len": wl.T, "parallelism": f"replicas{world}",
-            "l2": "inputs larger than L2 (no flush needed)"}
+            "l2": ("inputs larger than L2 (no flush needed)" if not wl.decode else
+                   "KV caches (1 GiB) larger than L2; each step gathers 42 rows per unit")}
 
 
 # ---- our arm -------------------------------------------------------------------
@@ -404,6 +432,131 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def run_ours_decode(args, rank, world, local_rank):
+    """Decode workloads: one new token per (layer, batch, head) at position
+    T - 1 against resident KV caches.  A step is one decode call over all
+    units; end to end, each step copies the new token's q, k and v rows in
+    (written into the caches at T - 1) and O and LSE out."""
+    import torch
+    import structured_sparse_attention_fibonacci_b200 as sa
+    from structured_sparse_attention_fibonacci_b200.inputs import WORKLOADS, make_decode_inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.workload]
+    wl_rank = wl.shrink(seed=wl.seed + 100000 * rank) if world > 1 else wl
+    q1_h, kc_h, vc_h = make_decode_inputs(wl_rank, pin=True)
+    q1, kc, vc = q1_h.to(dev), kc_h.to(dev), vc_h.to(dev)
+    alpha_h = wl.alpha().pin_memory()
+    alpha = alpha_h.to(dev)
+    pos = wl.T - 1
+    kw = dict(window=wl.window, sinks=wl.sinks, offsets=wl.offsets, rope_base=wl.rope_base)
+    o = torch.empty_like(q1)
+    lse = torch.empty(q1.shape[:3], dtype=torch.float32, device=dev)
+    units = wl.L * wl.B * wl.H
+    launches = [0]
+
+    def step():
+        sa.decode(q1, kc, vc, alpha, pos, out=o, lse=lse, **kw)
+        launches[0] += sa.last_launch_count()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.4)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches[0] = 0
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    gpu_launches = launches[0]
+    ms_max = max_over_ranks(e0.elapsed_time(e1), dev)
+    value = aggregate_throughput(units, world, args.steps, ms_max)
+
+    sa.trace_enable(True)
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    trace = sa.trace_read()
+    sa.trace_enable(False)
+    kernels = {n: {"ms_per_launch": t / c, "launches": c} for n, (t, c) in trace.items()}
+    elt = 2 if wl.dtype == torch.bfloat16 else 4
+    peak, peak_kind = measured_peaks()
+    bytes_launch = decode_bytes_per_token_head(wl, elt) * units
+    achieved = bytes_launch / (kernels["decode"]["ms_per_launch"] / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "decode", "achieved": achieved, "peak": peak,
+                "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                "alg_bytes_per_launch": bytes_launch,
+                "traffic": MEASURED_TRAFFIC.get(f"decode@{kernel_source_hash()}")}
+
+    # end to end: the new token's q, k, v rows in, O and LSE out, every step
+    kr_h = kc_h[:, :, :, pos].contiguous().pin_memory()
+    vr_h = vc_h[:, :, :, pos].contiguous().pin_memory()
+    o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    kr, vr = torch.empty_like(kr_h, device=dev), torch.empty_like(vr_h, device=dev)
+    h2d = (q1_h.numel() + kr_h.numel() + vr_h.numel()) * q1_h.element_size() + alpha_h.numel() * 4
+    d2h = o.numel() * o.element_size() + lse.numel() * 4
+
+    def e2e_step():
+        q1.copy_(q1_h, non_blocking=True)
+        kr.copy_(kr_h, non_blocking=True)
+        vr.copy_(vr_h, non_blocking=True)
+        alpha.copy_(alpha_h, non_blocking=True)
+        kc[:, :, :, pos].copy_(kr)
+        vc[:, :, :, pos].copy_(vr)
+        step()
+        o_h.copy_(o, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), dev)
+    e2e = {"value": aggregate_throughput(units, world, args.steps, e2e_ms), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": e2e_ms / args.steps}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(wl, args.cpu_budget_s)
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+                "config": workload_config(wl, world), "roofline": roofline,
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches, "clocks": clocks,
+                "kernels": kernels, "kernel_source": kernel_source_hash()}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -430,6 +583,9 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        from structured_sparse_attention_fibonacci_b200.inputs import WORKLOADS
+        if WORKLOADS[args.workload].decode:
+            return run_ours_decode(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:

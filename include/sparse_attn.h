@@ -165,6 +165,28 @@ sa_status sparse_attn_bwd_ctx(const sa_params* p, const void* q, const void* k, 
                               void* stream);
 
 /*
+ * Single-token decode with a KV cache: for every (layer, batch, head), the
+ * attention output of one new query at position `pos` against the cache rows
+ * 0..pos (the new token's own K/V row, at pos, included).  The result equals
+ * row `pos` of sparse_attn_fwd on the first pos + 1 rows with that query in
+ * row pos.  Source: the attended set, scaling and interpolation of
+ * "Depth-Staggered Fibonacci Spacing for Sparse Attention" (Methodology);
+ * the page measures inference latency for this gather (Results, efficiency).
+ *   p->T     : the cache length (rows allocated per unit); 0 <= pos < p->T
+ *   q        : device [L][B][H][D], unrotated (rotated at pos here)     (read)
+ *   k, v     : device [L][B][H][p->T][D] caches; only the rows the query
+ *              attends are read (window, sinks, offset rows; all <= pos)  (read)
+ *   alpha    : device fp32 [L]                                           (read)
+ *   o        : device [L][B][H][D], dtype p->dtype                     (written)
+ *   lse      : device fp32 [L][B][H] or NULL                           (written)
+ * Any dtype and head dim of sparse_attn_fwd; no workspace.  Returns
+ * SA_ERR_INVALID_ARG for pos outside [0, p->T).
+ */
+sa_status sparse_attn_decode(const sa_params* p, int32_t pos, const void* q, const void* k,
+                             const void* v, const float* alpha, void* o, float* lse,
+                             void* stream);
+
+/*
  * Forward that allocates no device memory.  The paper has no counterpart: this
  * entry point exists for callers that cannot let a library call cudaMalloc --
  * applications whose device memory belongs to a pooling allocator that must

@@ -59,6 +59,9 @@ class Oracle:
             geo.restype = ctypes.c_int
             geo.argtypes = [ctypes.c_float, ctypes.c_int32, ctypes.POINTER(ctypes.c_int64),
                             ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
+            dec = getattr(lib, "oracle_decode" + suffix)
+            dec.restype = ctypes.c_int
+            dec.argtypes = head + [ctypes.c_int64] + [P] * 5
             rope = getattr(lib, "oracle_rope" + suffix)
             rope.restype = None
             rope.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_double, P]
@@ -113,6 +116,27 @@ class Oracle:
             raise ValueError(f"oracle_bwd rejected its arguments (rc={rc})")
         return dq, dk, dv, dal
 
+    def decode(self, q1, k, v, alpha, pos, *, window, offsets=FIB15, sinks=0,
+               rope_base=10000.0, scale=0.0, precision="f64"):
+        """Single-token decode: q1 [L, B, H, D] at position pos against the
+        caches k, v [L, B, H, T, D] (rows 0..pos used).  Returns (O1, LSE1)."""
+        dt, ct = _np_dtype(precision)
+        q1, k, v = (_prep(x, dt) for x in (q1, k, v))
+        L, B, H, T, D = k.shape
+        assert v.shape == k.shape and q1.shape == (L, B, H, D)
+        al = _prep(alpha, np.float32).reshape(-1)
+        assert al.shape == (L,)
+        offs = np.ascontiguousarray(np.asarray(offsets, dtype=np.int32).reshape(-1))
+        o = np.empty_like(q1)
+        lse = np.empty((L, B, H), dtype=dt)
+        fn = getattr(self.lib, "oracle_decode_" + precision)
+        rc = fn(L, B, H, T, D, int(window), len(offs), _ptr(offs, ctypes.c_int32), int(sinks),
+                float(rope_base), float(scale), _ptr(al, ctypes.c_float), int(pos),
+                _ptr(q1, ct), _ptr(k, ct), _ptr(v, ct), _ptr(o, ct), _ptr(lse, ct))
+        if rc != 0:
+            raise ValueError(f"oracle_decode rejected its arguments (rc={rc})")
+        return o, lse
+
     def geometry(self, alpha, f):
         """(ok, lo, w, c) of one offset under the oracle's reading."""
         lo, w, c = ctypes.c_int64(), ctypes.c_double(), ctypes.c_int64()
@@ -145,6 +169,10 @@ def fwd(*a, **kw):
 
 def bwd(*a, **kw):
     return default().bwd(*a, **kw)
+
+
+def decode(*a, **kw):
+    return default().decode(*a, **kw)
 
 
 def geometry(alpha, f):

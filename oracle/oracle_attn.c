@@ -370,6 +370,73 @@ int FN(oracle_bwd)(int L, int B, int H, int T, int D, int W, int n_off,
   return err ? -2 : 0;
 }
 
+/*
+ * Single-token decode: for every unit, the output of one query q1 at
+ * position pos against K/V rows 0..pos (the attended set of query pos,
+ * "Attended set"; rows after pos are never touched).  Q1 and O1 are
+ * [L][B][H][D]; K and V are [L][B][H][T][D] with pos < T; LSE1 is
+ * [L][B][H] (may be NULL).  Each key row a member reads is rotated at its own
+ * position, one member at a time.
+ */
+int FN(oracle_decode)(int L, int B, int H, int T, int D, int W, int n_off,
+                      const int32_t* offsets, int S, double rope_base, double scale,
+                      const float* alpha, int64_t pos, const real* Q1, const real* K,
+                      const real* V, real* O1, real* LSE1) {
+  prob_t p = {L, B, H, T, D, W, n_off, S, rope_base, scale, offsets, alpha};
+  if (check(&p) || pos < 0 || pos >= T) return -1;
+  const double s = scale > 0 ? scale : 1.0 / sqrt((double)D);
+  const int n_slots = W + S + n_off;
+  const int64_t units = (int64_t)L * B * H;
+  int err = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
+  for (int64_t u = 0; u < units; ++u) {
+    const int l = (int)(u / ((int64_t)B * H));
+    geom_t g[ORACLE_MAX_OFFSETS];
+    for (int k = 0; k < n_off; ++k) g[k] = geometry(alpha[l], offsets[k]);
+    const real* Ku = K + u * (int64_t)T * D;
+    const real* Vu = V + u * (int64_t)T * D;
+    real* qh = (real*)malloc(sizeof(real) * D);
+    real* ka = (real*)malloc(sizeof(real) * D);
+    real* kb = (real*)malloc(sizeof(real) * D);
+    member_t* mb = (member_t*)malloc(sizeof(member_t) * (size_t)n_slots);
+    real* sc = (real*)malloc(sizeof(real) * (size_t)n_slots);
+    if (!qh || !ka || !kb || !mb || !sc) { err |= 1; goto done; }
+    rope_row(Q1 + u * D, pos, D, rope_base, qh);
+    for (int d = 0; d < D; ++d) qh[d] = (real)s * qh[d];
+    int n = members_of(pos, W, S, n_off, g, mb);
+    real mx = -INFINITY;
+    int any_nan = 0;
+    for (int m = 0; m < n; ++m) {
+      if (mb[m].nan_score) { sc[m] = (real)NAN; any_nan = 1; continue; }
+      rope_row(Ku + mb[m].a * D, mb[m].a, D, rope_base, ka);
+      real v = mb[m].wa * dot(qh, ka, D);
+      if (mb[m].b >= 0) {
+        rope_row(Ku + mb[m].b * D, mb[m].b, D, rope_base, kb);
+        v += mb[m].wb * dot(qh, kb, D);
+      }
+      sc[m] = v;
+      if (v > mx) mx = v;
+    }
+    real sum = 0;
+    for (int m = 0; m < n; ++m) {
+      sc[m] = any_nan ? (real)NAN : (real)exp((double)(sc[m] - mx));
+      sum += sc[m];
+    }
+    real* o = O1 + u * D;
+    for (int d = 0; d < D; ++d) o[d] = 0;
+    for (int m = 0; m < n; ++m) {
+      if (mb[m].nan_score) { for (int d = 0; d < D; ++d) o[d] = (real)NAN; continue; }
+      const real pm = sc[m] / sum;
+      gather_row(Vu, &mb[m], D, ka);
+      for (int d = 0; d < D; ++d) o[d] += pm * ka[d];
+    }
+    if (LSE1) LSE1[u] = any_nan ? (real)NAN : mx + (real)log((double)sum);
+  done:
+    free(qh); free(ka); free(kb); free(mb); free(sc);
+  }
+  return err ? -2 : 0;
+}
+
 /* Exposed for the pins: the geometry of one (alpha, f) and RoPE of one row. */
 int FN(oracle_geometry)(float alpha, int32_t f, int64_t* lo, double* w, int64_t* c) {
   geom_t g = geometry(alpha, f);

@@ -33,7 +33,8 @@ EXPORTED = ("sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_workspace_size",
             "sparse_attn_status_string", "sparse_attn_last_launch_count",
             "sparse_attn_trace_enable", "sparse_attn_trace_read", "sparse_attn_force_general",
             "sparse_attn_fwd_noalloc", "sparse_attn_device_error", "sparse_attn_select_forward",
-            "sparse_attn_context_size", "sparse_attn_fwd_train", "sparse_attn_bwd_ctx")
+            "sparse_attn_context_size", "sparse_attn_fwd_train", "sparse_attn_bwd_ctx",
+            "sparse_attn_decode")
 
 
 class SaParams(ctypes.Structure):
@@ -79,6 +80,8 @@ def lib():
         L.sparse_attn_last_launch_count.argtypes = []
         L.sparse_attn_force_general.restype = None
         L.sparse_attn_force_general.argtypes = [ctypes.c_int]
+        L.sparse_attn_decode.restype = ctypes.c_int
+        L.sparse_attn_decode.argtypes = [P, ctypes.c_int32, vp, vp, vp, fp, vp, fp, vp]
         L.sparse_attn_context_size.restype = ctypes.c_size_t
         L.sparse_attn_context_size.argtypes = [P]
         L.sparse_attn_fwd_train.restype = ctypes.c_int
@@ -238,6 +241,30 @@ def _fwd_train(q, k, v, alpha, *, window, offsets, sinks, rope_base, scale, out,
                                      _ptr(out), _ptr(lse), _ptr(context), context.numel(),
                                      _stream_handle(stream))
     _check("sparse_attn_fwd_train", st)
+    return out, lse
+
+
+def decode(q, k_cache, v_cache, alpha, pos, *, window, offsets=FIB15, sinks=0,
+           rope_base=10000.0, scale=0.0, out=None, lse=None, want_lse=True, stream=None):
+    """Single-token decode: q [L, B, H, D] at position pos against the caches
+    k_cache, v_cache [L, B, H, T_cache, D] (rows 0..pos hold the sequence,
+    row pos the new token).  Returns (O [L, B, H, D], LSE [L, B, H] or None)."""
+    shape = tuple(k_cache.shape)
+    dtype, dev = k_cache.dtype, k_cache.device
+    if tuple(q.shape) != shape[:3] + shape[4:]:
+        raise ValueError("q must be [L, B, H, D] matching the caches")
+    _check_tensors(shape, dtype, dev, k=k_cache, v=v_cache, alpha=alpha)
+    if q.dtype != dtype or not q.is_contiguous() or q.device != dev:
+        raise ValueError("q must be a contiguous tensor of the caches' dtype and device")
+    out = torch.empty_like(q) if out is None else out
+    if lse is None and want_lse:
+        lse = torch.empty(shape[:3], dtype=torch.float32, device=dev)
+    p = make_params(shape, dtype, window=window, offsets=offsets, sinks=sinks,
+                    rope_base=rope_base, scale=scale)
+    st = lib().sparse_attn_decode(ctypes.byref(p), int(pos), _ptr(q), _ptr(k_cache),
+                                  _ptr(v_cache), _ptr(alpha), _ptr(out), _ptr(lse),
+                                  _stream_handle(stream))
+    _check("sparse_attn_decode", st)
     return out, lse
 
 

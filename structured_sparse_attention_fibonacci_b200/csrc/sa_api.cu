@@ -233,6 +233,26 @@ sa_status sparse_attn_fwd(const sa_params* p, const void* q, const void* k, cons
   return SA_OK;
 }
 
+sa_status sparse_attn_decode(const sa_params* p, int32_t pos, const void* q, const void* k,
+                             const void* v, const float* alpha, void* o, float* lse,
+                             void* stream) {
+  sa::Problem pb;
+  sa_status s = build_problem(p, &pb);
+  if (s != SA_OK) return s;
+  if (pos < 0 || pos >= pb.T) return SA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !alpha || !o) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse && !aligned4(lse)) || !aligned4(alpha))
+    return SA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float2* rope = nullptr;
+  if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
+  if (sa::launch_decode(pb, pos, q, k, v, alpha, rope, o, lse, st) != cudaSuccess)
+    return SA_ERR_CUDA;
+  g_last_launches = 1;
+  return SA_OK;
+}
+
 size_t sparse_attn_context_size(const sa_params* p) {
   sa::Problem pb;
   if (build_problem(p, &pb) != SA_OK) return 0;

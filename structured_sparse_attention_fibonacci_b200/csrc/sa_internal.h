@@ -116,6 +116,10 @@ cudaError_t launch_reduce_dalpha(const float* part, int L, int per_layer, float*
                                  cudaStream_t st);
 
 cudaError_t launch_rope_table(float2* tab, int T, int D, double base, cudaStream_t st);
+// Single-token decode (sa_decode.cu): pb.T is the cache length, pos < pb.T.
+cudaError_t launch_decode(const Problem& pb, int pos, const void* q, const void* k, const void* v,
+                          const float* alpha, const float2* rope, void* o, float* lse,
+                          cudaStream_t st);
 cudaError_t launch_fwd_general(const Problem& pb, const FwdPtrs& a, cudaStream_t st, int* launches);
 cudaError_t launch_bwd_general(const Problem& pb, const BwdPtrs& a, cudaStream_t st, int* launches);
 

@@ -52,6 +52,7 @@ class Workload:
     alpha_kind: str            # "fixed", "linear", "coprime", "learned"
     seed: int                  # layer l uses seed + l (the tiny case: seed 0 for all)
     backward: bool = False
+    decode: bool = False       # one new token at position T - 1 against a T-row KV cache
     offsets: Tuple[int, ...] = FIB15
     rope_base: float = 10000.0
     note: str = ""
@@ -89,6 +90,11 @@ WORKLOADS = {
                               note="16 layers B=8 H=8 T=1024 d=64 bf16, W=12, learned alpha, fwd+bwd"),
     "long_sinks": Workload("long_sinks", 1, 1, 16, 32768, 64, 64, 4, torch.bfloat16, "fixed", 5000,
                            note="B=1 H=16 T=32768 d=64 bf16, W=64, 4 sinks, alpha=1"),
+    "decode_4k": Workload("decode_4k", 16, 8, 8, 4096, 64, 12, 0, torch.bfloat16, "linear", 6000,
+                          decode=True,
+                          note="single-token decode: 16 layers B=8 H=8 d=64 bf16, one new query "
+                               "at position 4095 against a 4096-row KV cache, W=12, linear "
+                               "stagger (the page measures inference latency of this gather)"),
 }
 
 
@@ -121,3 +127,22 @@ def make_dout(wl: Workload, seed: int = 77, device: Optional[str] = None):
     x = torch.randn((wl.L, wl.B, wl.H, wl.T, wl.D), generator=g, dtype=torch.float32)
     x = x.to(wl.dtype)
     return x if device is None else x.to(device)
+
+
+def make_decode_inputs(wl: Workload, device: Optional[str] = None, pin: bool = False):
+    """q [L, B, H, D] (the new token's queries) and the K, V caches
+    [L, B, H, T, D] of a decode workload.  Layer l draws q, then K, then V,
+    each N(0, 1) in fp32 from a CPU generator seeded with ``seed + l``, then
+    casts to the workload dtype."""
+    L, B, H, T, D = wl.L, wl.B, wl.H, wl.T, wl.D
+    q = torch.empty((L, B, H, D), dtype=wl.dtype, pin_memory=pin)
+    k = torch.empty((L, B, H, T, D), dtype=wl.dtype, pin_memory=pin)
+    v = torch.empty((L, B, H, T, D), dtype=wl.dtype, pin_memory=pin)
+    for l in range(L):
+        g = torch.Generator(device="cpu").manual_seed(wl.seed + l)
+        q[l].copy_(torch.randn((B, H, D), generator=g, dtype=torch.float32))
+        k[l].copy_(torch.randn((B, H, T, D), generator=g, dtype=torch.float32))
+        v[l].copy_(torch.randn((B, H, T, D), generator=g, dtype=torch.float32))
+    if device is not None:
+        q, k, v = q.to(device), k.to(device), v.to(device)
+    return q, k, v

@@ -270,6 +270,37 @@ def pin_fd_alpha(orc):
             assert abs(fd - dal[l]) <= 2e-3 * abs(fd) + 1e-6, (l, fd, dal[l])
 
 
+# -- single-token decode ------------------------------------------------------
+
+def pin_decode_dense_and_gather(orc):
+    """Decode at pos = the attended set of query pos: with W > pos and no
+    offsets it is row pos of plain dense causal attention; at alpha = 1 it is
+    row pos of the exact integer gather; rows after pos (NaN here) are never
+    read; and it matches row pos of the oracle forward with interpolation."""
+    L, B, H, T, D = 1, 1, 2, 70, 16
+    q, k, v = (_rand((L, B, H, T, D), s) for s in (70, 71, 72))
+    for pos in (0, 9, 40, 69):
+        kc, vc = k.copy(), v.copy()
+        kc[..., pos + 1:, :] = np.nan
+        vc[..., pos + 1:, :] = np.nan
+        q1 = q[..., pos, :]
+        o, lse = orc.decode(q1, kc, vc, [1.0], pos, window=T + 5, offsets=())
+        o_ref, lse_ref = dense_causal(q[..., :pos + 1, :], k[..., :pos + 1, :], v[..., :pos + 1, :])
+        _close(o, o_ref[..., pos, :], 1e-12, what=f"decode dense O pos={pos}")
+        _close(lse, lse_ref[..., pos], 1e-12, what=f"decode dense LSE pos={pos}")
+        o, lse = orc.decode(q1, kc, vc, [1.0], pos, window=6, sinks=2, offsets=FIB)
+        o_ref, lse_ref = integer_gather(q[..., :pos + 1, :], k[..., :pos + 1, :],
+                                        v[..., :pos + 1, :], window=6, sinks=2, dists=list(FIB))
+        _close(o, o_ref[..., pos, :], 1e-12, what=f"decode gather O pos={pos}")
+        _close(lse, lse_ref[..., pos], 1e-12, what=f"decode gather LSE pos={pos}")
+        for alpha in (0.63, 1.37):
+            o, lse = orc.decode(q1, kc, vc, [alpha], pos, window=5, sinks=1, offsets=FIB)
+            of, lf = orc.fwd(q[..., :pos + 1, :], k[..., :pos + 1, :], v[..., :pos + 1, :],
+                             [alpha], window=5, sinks=1, offsets=FIB)
+            _close(o, of[..., pos, :], 1e-12, what=f"decode vs forward alpha={alpha}")
+            _close(lse, lf[..., pos], 1e-12, what=f"decode vs forward LSE alpha={alpha}")
+
+
 ALL_PINS = [pin_geometry, pin_rope, pin_dense_limit, pin_integer_gather, pin_multiset,
             pin_softmax, pin_constant_v, pin_interp_continuity, pin_nan_geometry,
-            pin_fp32_build, pin_fd_inputs, pin_fd_alpha]
+            pin_fp32_build, pin_fd_inputs, pin_fd_alpha, pin_decode_dense_and_gather]

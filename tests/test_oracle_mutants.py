@@ -19,7 +19,10 @@ MUTANTS = [
     ("rope_freq", "double theta = pow(base, -2.0 * (double)j / (double)D);\n    double ang = (double)pos * theta;\n    real cs = (real)cos(ang), sn = (real)sin(ang);\n    real a = x[j], b = x[j + half];\n    out[j] = a * cs - b * sn;",
      "double theta = pow(base, -1.0 * (double)j / (double)D);\n    double ang = (double)pos * theta;\n    real cs = (real)cos(ang), sn = (real)sin(ang);\n    real a = x[j], b = x[j + half];\n    out[j] = a * cs - b * sn;"),
     ("rope_t_sign", "out[j] = a * cs + b * sn;", "out[j] = a * cs - b * sn;"),
-    ("lse_no_log", "mx + (real)log((double)sum)", "mx"),
+    ("lse_no_log", "LSE[u * T + i] = any_nan ? (real)NAN : mx + (real)log((double)sum)",
+     "LSE[u * T + i] = any_nan ? (real)NAN : mx"),
+    ("decode_lse_no_log", "LSE1[u] = any_nan ? (real)NAN : mx + (real)log((double)sum)",
+     "LSE1[u] = any_nan ? (real)NAN : mx"),
     ("geometry_round", "float fl = floorf(d);", "float fl = roundf(d);"),
     ("dq_no_scale", "dQ[base_off + i * D + d] *= (real)s;", "dQ[base_off + i * D + d] *= (real)1;"),
     ("dk_second_weight", "dKr[mb[m].b * D + d] += mb[m].wb * gs * qh[d];",
@@ -30,6 +33,11 @@ MUTANTS = [
     ("dalpha_sign", "t += gs * qh[d] * (kb[d] - ka[d])", "t += gs * qh[d] * (ka[d] - kb[d])"),
     ("dalpha_no_f", "dal += (real)g[mb[m].k].f * t;", "dal += t;"),
     ("dsigma_no_D", "const real gs = pm * (dp[m] - Dsum);", "const real gs = pm * dp[m];"),
+    ("decode_key_position", "rope_row(Ku + mb[m].a * D, mb[m].a, D, rope_base, ka);",
+     "rope_row(Ku + mb[m].a * D, pos, D, rope_base, ka);"),
+    ("decode_second_key_weight", "v += mb[m].wb * dot(qh, kb, D);", "v += mb[m].wa * dot(qh, kb, D);"),
+    ("decode_query_scale", "for (int d = 0; d < D; ++d) qh[d] = (real)s * qh[d];\n    int n = members_of(pos",
+     "for (int d = 0; d < D; ++d) qh[d] = qh[d];\n    int n = members_of(pos"),
 ]
 
 
