@@ -187,6 +187,23 @@ sa_status sparse_attn_decode(const sa_params* p, int32_t pos, const void* q, con
                              void* stream);
 
 /*
+ * Learned-alpha parametrisation.  The page trains "one free parameter theta
+ * per layer, initialised at alpha = 1" and constrains alpha to [0.5, 1.5]
+ * (Methodology: scaling; experimental variables); it does not give the map.
+ * The map used here: alpha = 0.5 + sigmoid(theta), so theta = 0 gives
+ * alpha = 1 and every theta lands inside the interval.
+ *   sparse_attn_alpha_from_theta: alpha[l] = 0.5 + 1 / (1 + exp(-theta[l]))
+ *   sparse_attn_dtheta: dtheta[l] = dalpha[l] * s (1 - s), s = sigmoid(theta[l])
+ *     (dalpha as written by sparse_attn_bwd / sparse_attn_bwd_ctx).
+ * theta, alpha, dalpha, dtheta: device fp32 [L], 4-byte aligned; fp32 math
+ * with the CUDA exponential.  One launch each on `stream`.
+ */
+sa_status sparse_attn_alpha_from_theta(int32_t L, const float* theta, float* alpha,
+                                       void* stream);
+sa_status sparse_attn_dtheta(int32_t L, const float* theta, const float* dalpha, float* dtheta,
+                             void* stream);
+
+/*
  * Forward that allocates no device memory.  The paper has no counterpart: this
  * entry point exists for callers that cannot let a library call cudaMalloc --
  * applications whose device memory belongs to a pooling allocator that must

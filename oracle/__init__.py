@@ -62,6 +62,12 @@ class Oracle:
             dec = getattr(lib, "oracle_decode" + suffix)
             dec.restype = ctypes.c_int
             dec.argtypes = head + [ctypes.c_int64] + [P] * 5
+            a_th = getattr(lib, "oracle_alpha_from_theta" + suffix)
+            a_th.restype = None
+            a_th.argtypes = [ctypes.c_int, P, P]
+            d_th = getattr(lib, "oracle_dtheta" + suffix)
+            d_th.restype = None
+            d_th.argtypes = [ctypes.c_int, P, P, P]
             rope = getattr(lib, "oracle_rope" + suffix)
             rope.restype = None
             rope.argtypes = [P, ctypes.c_int64, ctypes.c_int, ctypes.c_double, P]
@@ -136,6 +142,24 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"oracle_decode rejected its arguments (rc={rc})")
         return o, lse
+
+    def alpha_from_theta(self, theta, precision="f64"):
+        """alpha = 0.5 + sigmoid(theta) per layer (the learned-alpha map)."""
+        dt, ct = _np_dtype(precision)
+        th = _prep(theta, dt).reshape(-1)
+        out = np.empty_like(th)
+        getattr(self.lib, "oracle_alpha_from_theta_" + precision)(th.shape[0], _ptr(th, ct),
+                                                                  _ptr(out, ct))
+        return out
+
+    def dtheta(self, theta, dalpha, precision="f64"):
+        """Gradient to theta through alpha = 0.5 + sigmoid(theta)."""
+        dt, ct = _np_dtype(precision)
+        th, da = _prep(theta, dt).reshape(-1), _prep(dalpha, dt).reshape(-1)
+        out = np.empty_like(th)
+        getattr(self.lib, "oracle_dtheta_" + precision)(th.shape[0], _ptr(th, ct), _ptr(da, ct),
+                                                        _ptr(out, ct))
+        return out
 
     def geometry(self, alpha, f):
         """(ok, lo, w, c) of one offset under the oracle's reading."""

@@ -437,6 +437,24 @@ int FN(oracle_decode)(int L, int B, int H, int T, int D, int W, int n_off,
   return err ? -2 : 0;
 }
 
+/*
+ * Learned-alpha parametrisation ("Scaling": alpha is constrained to
+ * [0.5, 1.5]; "Experimental variables": the learned schedule has one free
+ * parameter theta per layer, initialised at alpha = 1).  The page gives no
+ * map; the reading taken is alpha = 0.5 + sigmoid(theta), and the gradient
+ * follows by the chain rule: dtheta = dalpha * sigmoid(theta) (1 - sigmoid(theta)).
+ */
+void FN(oracle_alpha_from_theta)(int L, const real* theta, real* alpha) {
+  for (int l = 0; l < L; ++l) alpha[l] = (real)(0.5 + 1.0 / (1.0 + exp(-(double)theta[l])));
+}
+
+void FN(oracle_dtheta)(int L, const real* theta, const real* dalpha, real* dtheta) {
+  for (int l = 0; l < L; ++l) {
+    const double s = 1.0 / (1.0 + exp(-(double)theta[l]));
+    dtheta[l] = (real)((double)dalpha[l] * s * (1.0 - s));
+  }
+}
+
 /* Exposed for the pins: the geometry of one (alpha, f) and RoPE of one row. */
 int FN(oracle_geometry)(float alpha, int32_t f, int64_t* lo, double* w, int64_t* c) {
   geom_t g = geometry(alpha, f);

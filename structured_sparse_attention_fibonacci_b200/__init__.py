@@ -34,7 +34,7 @@ EXPORTED = ("sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_workspace_size",
             "sparse_attn_trace_enable", "sparse_attn_trace_read", "sparse_attn_force_general",
             "sparse_attn_fwd_noalloc", "sparse_attn_device_error", "sparse_attn_select_forward",
             "sparse_attn_context_size", "sparse_attn_fwd_train", "sparse_attn_bwd_ctx",
-            "sparse_attn_decode")
+            "sparse_attn_decode", "sparse_attn_alpha_from_theta", "sparse_attn_dtheta")
 
 
 class SaParams(ctypes.Structure):
@@ -80,6 +80,10 @@ def lib():
         L.sparse_attn_last_launch_count.argtypes = []
         L.sparse_attn_force_general.restype = None
         L.sparse_attn_force_general.argtypes = [ctypes.c_int]
+        L.sparse_attn_alpha_from_theta.restype = ctypes.c_int
+        L.sparse_attn_alpha_from_theta.argtypes = [ctypes.c_int32, fp, fp, vp]
+        L.sparse_attn_dtheta.restype = ctypes.c_int
+        L.sparse_attn_dtheta.argtypes = [ctypes.c_int32, fp, fp, fp, vp]
         L.sparse_attn_decode.restype = ctypes.c_int
         L.sparse_attn_decode.argtypes = [P, ctypes.c_int32, vp, vp, vp, fp, vp, fp, vp]
         L.sparse_attn_context_size.restype = ctypes.c_size_t
@@ -242,6 +246,29 @@ def _fwd_train(q, k, v, alpha, *, window, offsets, sinks, rope_base, scale, out,
                                      _stream_handle(stream))
     _check("sparse_attn_fwd_train", st)
     return out, lse
+
+
+def alpha_from_theta(theta, alpha=None, stream=None):
+    """alpha = 0.5 + sigmoid(theta) per layer (the learned-alpha map); CUDA fp32 [L]."""
+    alpha = torch.empty_like(theta) if alpha is None else alpha
+    if theta.dtype != torch.float32 or alpha.dtype != torch.float32 or not theta.is_cuda:
+        raise ValueError("theta and alpha must be CUDA fp32 tensors")
+    st = lib().sparse_attn_alpha_from_theta(theta.numel(), _ptr(theta), _ptr(alpha),
+                                            _stream_handle(stream))
+    _check("sparse_attn_alpha_from_theta", st)
+    return alpha
+
+
+def dtheta(theta, dalpha, out=None, stream=None):
+    """Gradient to theta from dalpha through alpha = 0.5 + sigmoid(theta)."""
+    out = torch.empty_like(theta) if out is None else out
+    for t in (theta, dalpha, out):
+        if t.dtype != torch.float32 or not t.is_cuda:
+            raise ValueError("theta, dalpha and dtheta must be CUDA fp32 tensors")
+    st = lib().sparse_attn_dtheta(theta.numel(), _ptr(theta), _ptr(dalpha), _ptr(out),
+                                  _stream_handle(stream))
+    _check("sparse_attn_dtheta", st)
+    return out
 
 
 def decode(q, k_cache, v_cache, alpha, pos, *, window, offsets=FIB15, sinks=0,

@@ -253,6 +253,29 @@ sa_status sparse_attn_decode(const sa_params* p, int32_t pos, const void* q, con
   return SA_OK;
 }
 
+sa_status sparse_attn_alpha_from_theta(int32_t L, const float* theta, float* alpha,
+                                       void* stream) {
+  if (L < 1 || !theta || !alpha || !aligned4(theta) || !aligned4(alpha))
+    return SA_ERR_INVALID_ARG;
+  if (sa::launch_alpha_from_theta(L, theta, alpha, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return SA_ERR_CUDA;
+  g_last_launches = 1;
+  return SA_OK;
+}
+
+sa_status sparse_attn_dtheta(int32_t L, const float* theta, const float* dalpha, float* dtheta,
+                             void* stream) {
+  if (L < 1 || !theta || !dalpha || !dtheta || !aligned4(theta) || !aligned4(dalpha) ||
+      !aligned4(dtheta))
+    return SA_ERR_INVALID_ARG;
+  if (sa::launch_dtheta(L, theta, dalpha, dtheta, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return SA_ERR_CUDA;
+  g_last_launches = 1;
+  return SA_OK;
+}
+
 size_t sparse_attn_context_size(const sa_params* p) {
   sa::Problem pb;
   if (build_problem(p, &pb) != SA_OK) return 0;

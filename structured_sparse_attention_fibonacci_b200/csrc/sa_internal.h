@@ -116,6 +116,10 @@ cudaError_t launch_reduce_dalpha(const float* part, int L, int per_layer, float*
                                  cudaStream_t st);
 
 cudaError_t launch_rope_table(float2* tab, int T, int D, double base, cudaStream_t st);
+// Learned-alpha map (sa_theta.cu): alpha = 0.5 + sigmoid(theta) and its gradient.
+cudaError_t launch_alpha_from_theta(int L, const float* theta, float* alpha, cudaStream_t st);
+cudaError_t launch_dtheta(int L, const float* theta, const float* dalpha, float* dtheta,
+                          cudaStream_t st);
 // Single-token decode (sa_decode.cu): pb.T is the cache length, pos < pb.T.
 cudaError_t launch_decode(const Problem& pb, int pos, const void* q, const void* k, const void* v,
                           const float* alpha, const float2* rope, void* o, float* lse,

@@ -270,6 +270,42 @@ def pin_fd_alpha(orc):
             assert abs(fd - dal[l]) <= 2e-3 * abs(fd) + 1e-6, (l, fd, dal[l])
 
 
+# -- learned-alpha map ---------------------------------------------------------
+
+def pin_theta_map(orc):
+    """alpha = 0.5 + sigmoid(theta): theta = 0 is the initialisation alpha = 1,
+    theta = +-ln 3 gives 1.25 / 0.75 (sigmoid = 3/4, 1/4), alpha stays inside
+    [0.5, 1.5] and increases with theta; dtheta = dalpha * s (1 - s) equals a
+    central finite difference of the oracle's loss through alpha(theta)."""
+    th = np.array([0.0, np.log(3.0), -np.log(3.0), 40.0, -40.0, 0.3])
+    a = orc.alpha_from_theta(th)
+    _close(a[:3], [1.0, 1.25, 0.75], 1e-15, what="alpha(theta) closed forms")
+    assert (a >= 0.5).all() and (a <= 1.5).all()
+    grid = np.linspace(-8, 8, 101)
+    assert (np.diff(orc.alpha_from_theta(grid)) > 0).all()
+    # chain rule through the whole forward: theta chosen so alpha(theta) = FD_ALPHA
+    q, k, v, do = _fd_problem()
+    theta = -np.log(1.0 / (FD_ALPHA.astype(np.float64) - 0.5) - 1.0)
+    alpha = orc.alpha_from_theta(theta).astype(np.float32)
+    _close(alpha, FD_ALPHA, 1e-7, what="alpha(theta) round trip")
+    _, _, _, dal = orc.bwd(q, k, v, do, alpha, **FD_KW)
+    dth = orc.dtheta(theta, dal)
+    for l in range(2):
+        h = 1e-3
+        tp, tm = theta.copy(), theta.copy()
+        tp[l] += h
+        tm[l] -= h
+        ap = orc.alpha_from_theta(tp).astype(np.float32)
+        am = orc.alpha_from_theta(tm).astype(np.float32)
+        lp = float((orc.fwd(q, k, v, ap, **FD_KW)[0] * do).sum())
+        lm = float((orc.fwd(q, k, v, am, **FD_KW)[0] * do).sum())
+        # the fp32 rounding of alpha moves the step slightly: divide by the
+        # theta step that the rounded alphas correspond to
+        s = lambda x: 1.0 / (1.0 + np.exp(-x))
+        fd = (lp - lm) / (float(ap[l]) - float(am[l])) * (s(tp[l]) - s(tm[l])) / (2 * h)
+        assert abs(fd - dth[l]) <= 2e-3 * abs(fd) + 1e-6, (l, fd, dth[l])
+
+
 # -- single-token decode ------------------------------------------------------
 
 def pin_decode_dense_and_gather(orc):
@@ -303,4 +339,5 @@ def pin_decode_dense_and_gather(orc):
 
 ALL_PINS = [pin_geometry, pin_rope, pin_dense_limit, pin_integer_gather, pin_multiset,
             pin_softmax, pin_constant_v, pin_interp_continuity, pin_nan_geometry,
-            pin_fp32_build, pin_fd_inputs, pin_fd_alpha, pin_decode_dense_and_gather]
+            pin_fp32_build, pin_fd_inputs, pin_fd_alpha, pin_theta_map,
+            pin_decode_dense_and_gather]

@@ -33,6 +33,10 @@ MUTANTS = [
     ("dalpha_sign", "t += gs * qh[d] * (kb[d] - ka[d])", "t += gs * qh[d] * (ka[d] - kb[d])"),
     ("dalpha_no_f", "dal += (real)g[mb[m].k].f * t;", "dal += t;"),
     ("dsigma_no_D", "const real gs = pm * (dp[m] - Dsum);", "const real gs = pm * dp[m];"),
+    ("theta_map_offset", "alpha[l] = (real)(0.5 + 1.0 / (1.0 + exp(-(double)theta[l])));",
+     "alpha[l] = (real)(1.0 / (1.0 + exp(-(double)theta[l])));"),
+    ("dtheta_no_derivative", "dtheta[l] = (real)((double)dalpha[l] * s * (1.0 - s));",
+     "dtheta[l] = (real)((double)dalpha[l] * s);"),
     ("decode_key_position", "rope_row(Ku + mb[m].a * D, mb[m].a, D, rope_base, ka);",
      "rope_row(Ku + mb[m].a * D, pos, D, rope_base, ka);"),
     ("decode_second_key_weight", "v += mb[m].wb * dot(qh, kb, D);", "v += mb[m].wa * dot(qh, kb, D);"),
