@@ -241,7 +241,10 @@ def workload_config(wl, world):
     else:
         pass_ = "forward+backward" if wl.backward else "forward"
     return {"workload": wl.name, "L": wl.L, "B": wl.B, "H": wl.H, "T": wl.T, "D": wl.D,
-            "window": wl.window, "sinks": wl.sinks, "offsets": "fib15 (1..987)",
+            "window": wl.window, "sinks": wl.sinks,
+            "offsets": ("fib15 (1..987)" if tuple(wl.offsets) == (1, 2, 3, 5, 8, 13, 21, 34, 55, 89,
+                                                                  144, 233, 377, 610, 987)
+                        else list(wl.offsets)),
             "alpha": wl.alpha_kind, "pass": pass_,
             "global_batch": wl.B * world, "seq_len": wl.T, "parallelism": f"replicas{world}",
             "l2": ("inputs larger than L2 (no flush needed)" if not wl.decode else

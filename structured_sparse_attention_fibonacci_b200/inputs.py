@@ -90,6 +90,12 @@ WORKLOADS = {
                               note="16 layers B=8 H=8 T=1024 d=64 bf16, W=12, learned alpha, fwd+bwd"),
     "long_sinks": Workload("long_sinks", 1, 1, 16, 32768, 64, 64, 4, torch.bfloat16, "fixed", 5000,
                            note="B=1 H=16 T=32768 d=64 bf16, W=64, 4 sinks, alpha=1"),
+    "pi_skip": Workload("pi_skip", 16, 8, 8, 1024, 64, 5, 0, torch.bfloat16, "fixed", 7000,
+                        offsets=(16,),
+                        note="periodic skip in autoregressive form: local window of the "
+                             "current and 4 previous keys plus one skip to i - 16 (k = 4, "
+                             "pi = 16, the best setting of the pi-Attention page), 16 layers "
+                             "B=8 H=8 T=1024 d=64 bf16"),
     "decode_4k": Workload("decode_4k", 16, 8, 8, 4096, 64, 12, 0, torch.bfloat16, "linear", 6000,
                           decode=True,
                           note="single-token decode: 16 layers B=8 H=8 d=64 bf16, one new query "

@@ -142,6 +142,7 @@ FAST = [
     ("fast_w1", (1, 1, 2, 200, 64), 1, 0, [1.37], FIB15),
     ("fast_w7_odd", (2, 1, 1, 300, 64), 7, 3, [0.61, 1.44], FIB15),
     ("fast_long_1500", (1, 1, 1, 1700, 64), 12, 0, [1.5], FIB15),
+    ("fast_pi_skip", (2, 1, 2, 300, 64), 5, 0, [1.0, 1.0], (16,)),
 ]
 
 
