@@ -136,12 +136,13 @@ sa_status sparse_attn_bwd(const sa_params* p, const void* q, const void* k, cons
  * (the paper has no counterpart; its training runs a forward and a backward
  * per step): the forward keeps, in the caller's `context` buffer,
  *   - the RoPE-rotated keys (fp16 of RoPE(K) / 256, [L][B][H][T][D]),
+ *   - the rotated, scaled queries (fp16 of RoPE(Q) * scale / 256, same layout),
  *   - every member's softmax probability (window lags 0..W-1 unfolded, sinks,
  *     offsets in the order of p->offsets sorted ascending), fp32
  *     [L*B*H][W+S+n_offsets][T],
  *   - every offset's row-score difference score(row i-lo-1) - score(row i-lo),
  *     fp32 [L*B*H][n_offsets][T],
- * and sparse_attn_bwd_ctx then skips the score pass and the key rotation.
+ * and sparse_attn_bwd_ctx then skips the score pass and both rotation pre-passes.
  * Results equal sparse_attn_fwd / sparse_attn_bwd up to fp32 rounding order.
  *
  * sparse_attn_context_size: bytes of the context for these params; 0 when

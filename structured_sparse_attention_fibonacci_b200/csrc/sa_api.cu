@@ -305,7 +305,8 @@ sa_status sparse_attn_fwd_train(const sa_params* p, const void* q, const void* k
   int launches = 0;
   if (sa::launch_fwd_fast(pb, a, cb + cl.khat_off, st, &launches,
                           reinterpret_cast<float*>(cb + cl.p_off),
-                          reinterpret_cast<float*>(cb + cl.dt_off)) != cudaSuccess)
+                          reinterpret_cast<float*>(cb + cl.dt_off), cb + cl.qhat_off) !=
+      cudaSuccess)
     return SA_ERR_CUDA;
   g_last_launches = launches;
   return SA_OK;

@@ -47,6 +47,7 @@ struct FastArgs {
   unsigned* err;
   float* save_p;                       // SAVE: [units][W+S+n_off][T] member probabilities
   float* save_dt;                      // SAVE: [units][n_off][T] row-score differences
+  __half* save_q;                      // SAVE: [units][T][64] fp16 of RoPE(Q) * scale / 256
 };
 
 enum : int { kFar = 0, kNear = 1, kDead = 2 };
@@ -267,6 +268,24 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
     }
   }
   const int off0 = half0_off(c, par), d1 = half1_off(c, par) - off0;
+  if (SAVE) {
+    // the backward's rotated, scaled queries: q holds RoPE(Q) * scale * 256
+    const int h0 = c + 4 * par, h1 = c + 4 - 4 * par;
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) {
+      const int i = ig + qq;
+      if (i >= T) continue;
+      float y0[8], y1[8];
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        y0[h] = q[qq][h] * (kKeyStage * kKeyStage);
+        y1[h] = q[qq][h + 8] * (kKeyStage * kKeyStage);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(a.save_q + ub + (size_t)i * kD);
+      dst[h0] = pack8_h(y0);
+      dst[h1] = pack8_h(y1);
+    }
+  }
 
   const int lr = 4 * gid + c;                  // this lane's query, tile-local
   const int i_own = ig + c;                    // ... and its position
@@ -512,7 +531,7 @@ size_t fast_fwd_workspace(const Problem& pb) {
 }
 
 cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& p, void* keys_ws, cudaStream_t st,
-                            int* launches, float* save_p, float* save_dt) {
+                            int* launches, float* save_p, float* save_dt, void* save_q) {
   FastArgs a = {};
   a.B = pb.B; a.H = pb.H; a.T = pb.T; a.W = pb.W; a.n_off = pb.n_off; a.S = pb.S;
   a.n_tiles = (pb.T + kFastM - 1) / kFastM;
@@ -524,7 +543,7 @@ cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& p, void* keys_ws, 
   a.v = reinterpret_cast<const __nv_bfloat16*>(p.v);
   a.alpha = p.alpha; a.rope = p.rope;
   a.o = reinterpret_cast<__nv_bfloat16*>(p.o); a.lse = p.lse;
-  a.save_p = save_p; a.save_dt = save_dt;
+  a.save_p = save_p; a.save_dt = save_dt; a.save_q = reinterpret_cast<__half*>(save_q);
   cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&a.err), g_fwd_err);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((long long)pb.units() * a.n_tiles);
@@ -544,7 +563,8 @@ cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& p, void* keys_ws, 
       return e;
     *launches += 1;
     a.k = keys_ws;
-    e = (save_p && save_dt) ? launch(k_fwd_fast<true, true>) : launch(k_fwd_fast<true, false>);
+    e = (save_p && save_dt && save_q) ? launch(k_fwd_fast<true, true>)
+                                      : launch(k_fwd_fast<true, false>);
   } else {
     a.k = p.k;
     e = launch(k_fwd_fast<false, false>);

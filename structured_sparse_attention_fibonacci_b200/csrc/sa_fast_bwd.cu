@@ -889,7 +889,7 @@ cudaError_t launch_bwd_fast(const Problem& pb, const BwdPtrs& p, cudaStream_t st
   const CtxLayout CL = ctx_layout(pb);
   const char* cb = reinterpret_cast<const char*>(ctx);
   void* khat = ctx ? const_cast<char*>(cb + CL.khat_off) : ws + L.khat_off;
-  void* qhat = ws + L.qhat_off;
+  void* qhat = ctx ? const_cast<char*>(cb + CL.qhat_off) : ws + L.qhat_off;
   if (ctx) {
     a.ctx_p = reinterpret_cast<const float*>(cb + CL.p_off);
     a.ctx_dt = reinterpret_cast<const float*>(cb + CL.dt_off);
@@ -908,8 +908,8 @@ cudaError_t launch_bwd_fast(const Problem& pb, const BwdPtrs& p, cudaStream_t st
   if (!ctx && (e = launch_rope_rows(p.k, p.rope, pb.T, n_rows, kKeyStage, khat, st,
                                     "rope_keys")) != cudaSuccess)
     return e;
-  if ((e = launch_rope_rows(p.q, p.rope, pb.T, n_rows, pb.scale * kKeyStage, qhat, st,
-                            "rope_queries")) != cudaSuccess)
+  if (!ctx && (e = launch_rope_rows(p.q, p.rope, pb.T, n_rows, pb.scale * kKeyStage, qhat, st,
+                                    "rope_queries")) != cudaSuccess)
     return e;
   auto kq = ctx ? k_bwd_q_fast<true> : k_bwd_q_fast<false>;
   if ((e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -930,7 +930,7 @@ cudaError_t launch_bwd_fast(const Problem& pb, const BwdPtrs& p, cudaStream_t st
   if ((e = launch_reduce_dalpha(a.dal_part, pb.L, pb.B * pb.H * L.n_tiles, p.dalpha, st)) !=
       cudaSuccess)
     return e;
-  *launches += ctx ? 4 : 5;
+  *launches += ctx ? 3 : 5;
   return cudaSuccess;
 }
 

@@ -60,11 +60,13 @@ void trace_mark(const char* kernel, cudaStream_t st, bool begin);
 bool fast_fwd_supported(const Problem& pb);
 size_t fast_fwd_smem(const Problem& pb, int* ring_rows, int* sc_stride);
 size_t fast_fwd_workspace(const Problem& pb);
-// With save_p / save_dt (the training context) it also stores every member's
-// probability ([units][W+S+n_off][T]) and every offset's row-score difference
-// ([units][n_off][T]), fp32, for sparse_attn_bwd_ctx.
+// With save_p / save_dt / save_q (the training context) it also stores every
+// member's probability ([units][W+S+n_off][T]) and every offset's row-score
+// difference ([units][n_off][T]), fp32, and the rotated, scaled queries
+// (fp16 of RoPE(Q) * scale / 256, [units][T][64]) for sparse_attn_bwd_ctx.
 cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& a, void* keys_ws, cudaStream_t st,
-                            int* launches, float* save_p = nullptr, float* save_dt = nullptr);
+                            int* launches, float* save_p = nullptr, float* save_dt = nullptr,
+                            void* save_q = nullptr);
 // Tensor-core bf16 / D=64 forward (sa_fwd_tc.cu); keys_ws as for the staged
 // forward (fast_fwd_workspace bytes, required).
 bool tc_fwd_supported(const Problem& pb);
@@ -98,14 +100,15 @@ cudaError_t launch_bwd_fast(const Problem& pb, const BwdPtrs& a, cudaStream_t st
 
 // Training context layout (shared by sa_api.cu and the kernels' launchers).
 struct CtxLayout {
-  size_t khat_off, p_off, dt_off, total;
+  size_t khat_off, qhat_off, p_off, dt_off, total;
 };
 inline CtxLayout ctx_layout(const Problem& pb) {
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   const size_t units = (size_t)pb.units(), T = (size_t)pb.T;
   CtxLayout c;
   c.khat_off = 0;
-  c.p_off = up(units * T * 64 * 2);
+  c.qhat_off = up(units * T * 64 * 2);
+  c.p_off = c.qhat_off + up(units * T * 64 * 2);
   c.dt_off = c.p_off + up(units * (size_t)(pb.W + pb.S + pb.n_off) * T * sizeof(float));
   c.total = c.dt_off + up(units * (size_t)pb.n_off * T * sizeof(float));
   return c;

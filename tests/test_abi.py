@@ -124,7 +124,7 @@ def test_context_size_and_validation(lib):
     f = lambda p: lib.sparse_attn_context_size(ctypes.byref(p))
     units, T = 16 * 8 * 8, 1024
     n = f(_p())
-    assert n >= units * T * (64 * 2 + 4 * (12 + 15 + 15))
+    assert n >= units * T * (2 * 64 * 2 + 4 * (12 + 15 + 15))
     assert f(_p(dtype=torch.float32)) == 0
     assert f(_p(shape=(1, 1, 1, 64, 32))) == 0
     dummy = ctypes.c_void_p(1 << 20)     # never dereferenced: validation comes first
