@@ -236,21 +236,33 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
         for (int mt = 0; mt < 2; ++mt) {
           const int qb = i0 + 32 * warp + 16 * mt, ql = 32 * warp + 16 * mt;
           const int rb = qb - og.lo - (two ? 1 : 0);
-          // three n tiles (24 rows; the third only matters when w != 0),
-          // loads first, then the three accumulator chains interleaved
+          // three n tiles (24 rows) when w != 0, two when w == 0; loads
+          // first, then the accumulator chains interleaved
           uint32_t b[3][2][4];
-#pragma unroll
-          for (int nt = 0; nt < 3; ++nt) qk_load(ring_u32, RB, rb + 8 * nt, lane, b[nt]);
           float cc[3][4];
 #pragma unroll
           for (int nt = 0; nt < 3; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) cc[nt][e] = 0.f;
+          if (two) {
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
+            for (int nt = 0; nt < 3; ++nt) qk_load(ring_u32, RB, rb + 8 * nt, lane, b[nt]);
 #pragma unroll
-            for (int nt = 0; nt < 3; ++nt)
-              mma_f16(cc[nt], aq[mt][ks], b[nt][ks >> 1][2 * (ks & 1)], b[nt][ks >> 1][2 * (ks & 1) + 1]);
+            for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+              for (int nt = 0; nt < 3; ++nt)
+                mma_f16(cc[nt], aq[mt][ks], b[nt][ks >> 1][2 * (ks & 1)],
+                        b[nt][ks >> 1][2 * (ks & 1) + 1]);
+          } else {                               // w == 0: row a only, two n tiles
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) qk_load(ring_u32, RB, rb + 8 * nt, lane, b[nt]);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+              for (int nt = 0; nt < 2; ++nt)
+                mma_f16(cc[nt], aq[mt][ks], b[nt][ks >> 1][2 * (ks & 1)],
+                        b[nt][ks >> 1][2 * (ks & 1) + 1]);
+          }
           const float (&c0)[4] = cc[0];
           const float (&c1)[4] = cc[1];
           const float (&c2)[4] = cc[2];
