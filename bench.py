@@ -36,10 +36,13 @@ FALLBACK_HBM_GBS = 6650.0
 #   bwd key  : read Q, K, V, dO, LSE, D; write dK, dV
 #   RoPE pre-pass (rope_keys / rope_queries): read K (or Q), write it rotated
 # (the whole backward: Q, K, V, O, dO, dQ, dK, dV and LSE = 1028 B)
-def alg_bytes_per_token_head(kernel, D, elt):
+def alg_bytes_per_token_head(kernel, D, elt, context=0):
+    """Bytes a kernel must move per token-head: every input row read once and
+    every output written once.  ``context``: bytes per token-head the saving
+    forward also writes into the training context (0 without one)."""
     row = D * elt
     if kernel.startswith("fwd"):
-        return 4 * row + 4
+        return 4 * row + 4 + context
     if kernel.startswith("bwd_q"):
         return 6 * row + 8
     if kernel.startswith("bwd_kv"):
@@ -57,13 +60,19 @@ def decode_bytes_per_token_head(wl, elt):
     return 2 * row + 4 + 2 * rows * row
 
 
-# dram__bytes_read.sum + dram__bytes_write.sum per token-head from the ncu
-# captures summarised under profiles/, keyed by kernel and the hash of the
-# kernel sources they were taken on; a changed source reports null.
+# dram__bytes_read.sum + dram__bytes_write.sum per token-head (per
+# (layer, batch, head) for decode) from the ncu captures summarised under
+# profiles/, keyed by workload, kernel and the hash of the kernel sources they
+# were taken on; a changed source reports null.
 MEASURED_TRAFFIC = {
-    # profiles/staged_kernels_learned_train.md: 579.8 + 238.6 MB per launch of
-    # the context-mode query side over 1048576 token-heads
-    "bwd_q_fast@20d57b6d526b": 780.5,
+    # profiles/staged_kernels_learned_train.md (one launch, 1048576 token-heads)
+    "learned_train/bwd_q_fast@cb35362de4bc": 779.3,
+    # profiles/forward_and_decode_traffic.md
+    "paper_fwd/fwd_fast@cb35362de4bc": 495.2,
+    "extrap_4x/fwd_fast@cb35362de4bc": 497.0,
+    "pi_skip/fwd_fast@cb35362de4bc": 492.5,
+    "long_sinks/fwd_tc@cb35362de4bc": 508.7,
+    "decode_4k/decode@cb35362de4bc": 8145.5,
 }
 
 
@@ -334,17 +343,20 @@ def run_ours(args, rank, world, local_rank):
     dominant = max(kernels, key=lambda n: kernels[n]["ms_per_launch"] * kernels[n]["launches"])
     elt = 2 if wl.dtype == torch.bfloat16 else 4
     peak, peak_kind = measured_peaks()
-    per_th = alg_bytes_per_token_head(dominant, wl.D, elt)
+    # the training context per token-head: fp32 probabilities of every
+    # member, fp32 row-score differences per offset, the fp16 rotated query
+    ctx_th = ((wl.window + wl.sinks + 2 * len(wl.offsets)) * 4 + wl.D * 2) if wl.backward else 0
+    per_th = alg_bytes_per_token_head(dominant, wl.D, elt, ctx_th)
     bytes_launch = per_th * wl.token_heads
     achieved = bytes_launch / (kernels[dominant]["ms_per_launch"] / 1e3) / 1e9
-    key = f"{dominant}@{kernel_source_hash()}"
+    key = f"{wl.name}/{dominant}@{kernel_source_hash()}"
     traffic = MEASURED_TRAFFIC.get(key)
     roofline = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
                 "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                 "alg_bytes_per_launch": bytes_launch,
                 "traffic": traffic * wl.token_heads if traffic is not None else None}
     for n, kk in kernels.items():
-        b = alg_bytes_per_token_head(n, wl.D, elt) * wl.token_heads
+        b = alg_bytes_per_token_head(n, wl.D, elt, ctx_th) * wl.token_heads
         kk["alg_GBps"] = b / (kk["ms_per_launch"] / 1e3) / 1e9 if b else None
 
     # End to end through the public API: every step copies its inputs in from
@@ -509,7 +521,10 @@ def run_ours_decode(args, rank, world, local_rank):
     roofline = {"bound": "hbm", "kernel": "decode", "achieved": achieved, "peak": peak,
                 "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                 "alg_bytes_per_launch": bytes_launch,
-                "traffic": MEASURED_TRAFFIC.get(f"decode@{kernel_source_hash()}")}
+                "traffic": None}
+    traffic = MEASURED_TRAFFIC.get(f"{wl.name}/decode@{kernel_source_hash()}")
+    if traffic is not None:
+        roofline["traffic"] = traffic * units
 
     # end to end: the new token's q, k, v rows in, O and LSE out, every step
     kr_h = kc_h[:, :, :, pos].contiguous().pin_memory()
