@@ -51,10 +51,10 @@ class Oracle:
                                          ctypes.POINTER(ctypes.c_float)]
             fwd = getattr(lib, "oracle_fwd" + suffix)
             fwd.restype = ctypes.c_int
-            fwd.argtypes = head + [P] * 6
+            fwd.argtypes = head + [P] * 7
             bwd = getattr(lib, "oracle_bwd" + suffix)
             bwd.restype = ctypes.c_int
-            bwd.argtypes = head + [P] * 8
+            bwd.argtypes = head + [P] * 10
             geo = getattr(lib, "oracle_geometry" + suffix)
             geo.restype = ctypes.c_int
             geo.argtypes = [ctypes.c_float, ctypes.c_int32, ctypes.POINTER(ctypes.c_int64),
@@ -75,8 +75,10 @@ class Oracle:
         self.path = path
 
     def fwd(self, q, k, v, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0,
-            scale=0.0, precision="f64", want_probs=False):
-        """Forward.  q, k, v: [L, B, H, T, D] (upcast); alpha: [L] fp32 values.
+            scale=0.0, precision="f64", want_probs=False, beta=None):
+        """Forward.  q, k, v: [L, B, H, T, D] (upcast); alpha: [L] fp32 values;
+        beta: optional [L, B, H, T] log-prior added to every offset member's
+        score of each query (None: no prior).
 
         Returns (O, LSE) or (O, LSE, P), P [L, B, H, T, W+S+n_off] holding each
         member's softmax weight in a fixed slot (window t, sink s, offset k),
@@ -93,18 +95,21 @@ class Oracle:
         lse = np.empty((L, B, H, T), dtype=dt)
         n_slots = window + sinks + len(offs)
         p = np.empty((L, B, H, T, n_slots), dtype=dt) if want_probs else None
+        bt = _prep(beta, dt).reshape(L, B, H, T) if beta is not None else None
         fn = getattr(self.lib, "oracle_fwd_" + precision)
         rc = fn(L, B, H, T, D, int(window), len(offs), _ptr(offs, ctypes.c_int32), int(sinks),
                 float(rope_base), float(scale), _ptr(al, ctypes.c_float),
                 _ptr(q, ct), _ptr(k, ct), _ptr(v, ct), _ptr(o, ct), _ptr(lse, ct),
-                _ptr(p, ct) if p is not None else None)
+                _ptr(p, ct) if p is not None else None,
+                _ptr(bt, ct) if bt is not None else None)
         if rc != 0:
             raise ValueError(f"oracle_fwd rejected its arguments (rc={rc})")
         return (o, lse, p) if want_probs else (o, lse)
 
     def bwd(self, q, k, v, dout, alpha, *, window, offsets=FIB15, sinks=0,
-            rope_base=10000.0, scale=0.0, precision="f64"):
-        """Backward for upstream dO: returns (dQ, dK, dV, dalpha[L])."""
+            rope_base=10000.0, scale=0.0, precision="f64", beta=None):
+        """Backward for upstream dO: returns (dQ, dK, dV, dalpha[L]), and with
+        a log-prior beta [L, B, H, T] also dbeta: (dQ, dK, dV, dalpha, dbeta)."""
         dt, ct = _np_dtype(precision)
         q, k, v, dout = (_prep(x, dt) for x in (q, k, v, dout))
         L, B, H, T, D = q.shape
@@ -113,14 +118,18 @@ class Oracle:
         offs = np.ascontiguousarray(np.asarray(offsets, dtype=np.int32).reshape(-1))
         dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
         dal = np.empty((L,), dtype=dt)
+        bt = _prep(beta, dt).reshape(L, B, H, T) if beta is not None else None
+        dbt = np.empty((L, B, H, T), dtype=dt) if beta is not None else None
         fn = getattr(self.lib, "oracle_bwd_" + precision)
         rc = fn(L, B, H, T, D, int(window), len(offs), _ptr(offs, ctypes.c_int32), int(sinks),
                 float(rope_base), float(scale), _ptr(al, ctypes.c_float),
                 _ptr(q, ct), _ptr(k, ct), _ptr(v, ct), _ptr(dout, ct),
-                _ptr(dq, ct), _ptr(dk, ct), _ptr(dv, ct), _ptr(dal, ct))
+                _ptr(dq, ct), _ptr(dk, ct), _ptr(dv, ct), _ptr(dal, ct),
+                _ptr(bt, ct) if bt is not None else None,
+                _ptr(dbt, ct) if dbt is not None else None)
         if rc != 0:
             raise ValueError(f"oracle_bwd rejected its arguments (rc={rc})")
-        return dq, dk, dv, dal
+        return (dq, dk, dv, dal, dbt) if beta is not None else (dq, dk, dv, dal)
 
     def decode(self, q1, k, v, alpha, pos, *, window, offsets=FIB15, sinks=0,
                rope_base=10000.0, scale=0.0, precision="f64"):

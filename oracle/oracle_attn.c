@@ -25,6 +25,16 @@
  *   An offset with d_k outside [0, 2^24) (alpha negative, NaN, or huge) has
  *   no defined row: its score is NaN, so the query's outputs become NaN.
  *
+ * Optional additive log-prior on the offset members.  "pi-Attention: Periodic
+ * Sparse Transformers for Efficient Long-Context Modeling" (Core components,
+ * dynamic adaptive fusion) merges its local and skip logits into one softmax
+ * by adding a log-prior in the log domain.  Softmax ignores a shift common to
+ * all of a query's members, so the two per-query priors act only through
+ * their difference: here one value beta[i] per query is added to the score
+ * of every offset member of query i.  The window and the sinks get 0.  The
+ * gradient is dbeta[i] = sum over those offset members of dLoss/dscore.
+ * beta is [L][B][H][T] and may be NULL, meaning zero.
+ *
  * This file is compiled twice: with ORACLE_REAL=double / ORACLE_SUFFIX=_f64
  * (parity reference and finite differences) and with ORACLE_REAL=float /
  * ORACLE_SUFFIX=_f32 (the plain fp32 CPU baseline).  RoPE angles and their
@@ -186,11 +196,12 @@ static void rotate_unit(const real* K, int64_t T, int D, double base, real* Kr) 
  * Forward.  O[L][B][H][T][D], LSE[L][B][H][T] (may be NULL), and optionally
  * P[L][B][H][T][W+S+n_off]: each member's softmax weight in its fixed slot
  * (window t, then sink s, then offset k), 0 for members that do not exist.
+ * beta (may be NULL): the per-query log-prior on the offset members.
  */
 int FN(oracle_fwd)(int L, int B, int H, int T, int D, int W, int n_off,
                    const int32_t* offsets, int S, double rope_base, double scale,
                    const float* alpha, const real* Q, const real* K, const real* V,
-                   real* O, real* LSE, real* P) {
+                   real* O, real* LSE, real* P, const real* beta) {
   prob_t p = {L, B, H, T, D, W, n_off, S, rope_base, scale, offsets, alpha};
   if (check(&p)) return -1;
   const double s = scale > 0 ? scale : 1.0 / sqrt((double)D);
@@ -221,6 +232,7 @@ int FN(oracle_fwd)(int L, int B, int H, int T, int D, int W, int n_off,
         if (mb[m].nan_score) { sc[m] = (real)NAN; any_nan = 1; continue; }
         gather_row(Kr, &mb[m], D, row);
         sc[m] = dot(qh, row, D);
+        if (beta && mb[m].kind == 2) sc[m] += beta[u * T + i];   /* log-prior */
         if (sc[m] > mx) mx = sc[m];
       }
       real sum = 0;
@@ -258,11 +270,14 @@ int FN(oracle_fwd)(int L, int B, int H, int T, int D, int W, int n_off,
  * weight w = alpha*f - floor(alpha*f), dw/dalpha = f ("Implementation": the
  * interpolation exists so that gradients reach alpha).  floor() is held fixed
  * (the right derivative at integer d); a second row i-lo-1 < 0 contributes 0.
+ * beta (may be NULL): the forward's log-prior; dbeta (may be NULL) receives
+ * its gradient [L][B][H][T].
  */
 int FN(oracle_bwd)(int L, int B, int H, int T, int D, int W, int n_off,
                    const int32_t* offsets, int S, double rope_base, double scale,
                    const float* alpha, const real* Q, const real* K, const real* V,
-                   const real* dO, real* dQ, real* dK, real* dV, real* dalpha) {
+                   const real* dO, real* dQ, real* dK, real* dV, real* dalpha,
+                   const real* beta, real* dbeta) {
   prob_t p = {L, B, H, T, D, W, n_off, S, rope_base, scale, offsets, alpha};
   if (check(&p)) return -1;
   const double s = scale > 0 ? scale : 1.0 / sqrt((double)D);
@@ -297,6 +312,8 @@ int FN(oracle_bwd)(int L, int B, int H, int T, int D, int W, int n_off,
         for (int64_t e = 0; e < (int64_t)T * D; ++e)
           dQ[base_off + e] = dK[base_off + e] = dVu[e] = (real)NAN;
         dal_unit[u] = (real)NAN;
+        if (dbeta)
+          for (int64_t i = 0; i < T; ++i) dbeta[u * T + i] = (real)NAN;
         goto done;
       }
     }
@@ -313,6 +330,7 @@ int FN(oracle_bwd)(int L, int B, int H, int T, int D, int W, int n_off,
         gather_row(Kr, &mb[m], D, krow + m * D);
         gather_row(Vu, &mb[m], D, vrow + m * D);
         sc[m] = dot(qh, krow + m * D, D);
+        if (beta && mb[m].kind == 2) sc[m] += beta[u * T + i];   /* log-prior */
         if (sc[m] > mx) mx = sc[m];
       }
       real sum = 0;
@@ -322,9 +340,11 @@ int FN(oracle_bwd)(int L, int B, int H, int T, int D, int W, int n_off,
       real Dsum = 0;
       for (int m = 0; m < n; ++m) { dp[m] = dot(go, vrow + m * D, D); Dsum += sc[m] * dp[m]; }
       for (int d = 0; d < D; ++d) dqh[d] = 0;
+      real dbet = 0;    /* d score of each offset member, summed: d beta_i */
       for (int m = 0; m < n; ++m) {
         const real pm = sc[m];
         const real gs = pm * (dp[m] - Dsum);
+        if (mb[m].kind == 2) dbet += gs;
         const real* kr = krow + m * D;
         for (int d = 0; d < D; ++d) dqh[d] += gs * kr[d];
         /* scatter onto the rows the member read */
@@ -354,6 +374,7 @@ int FN(oracle_bwd)(int L, int B, int H, int T, int D, int W, int n_off,
       /* q_hat = s * R_i Q_i  ->  dQ_i = s * R_i^T dq_hat */
       rope_row_t(dqh, i, D, rope_base, dQ + base_off + i * D);
       for (int d = 0; d < D; ++d) dQ[base_off + i * D + d] *= (real)s;
+      if (dbeta) dbeta[u * T + i] = dbet;
     }
     for (int64_t j = 0; j < T; ++j) rope_row_t(dKr + j * D, j, D, rope_base, dK + base_off + j * D);
     dal_unit[u] = dal;

@@ -14,6 +14,9 @@ shows up as a disagreement.
   multiset_bias     -- log-multiplicity bias that turns dense causal attention
                        into the sparse attended set when every distance is an
                        integer (duplicates counted).
+  prior_bias        -- the same with a per-query log-prior on the offset
+                       members: key j of query i weighs
+                       (local multiplicity) + (offset multiplicity) * e^beta_i.
 """
 import numpy as np
 
@@ -95,3 +98,26 @@ def multiset_bias(T, *, window, dists, sinks=0):
                 cnt[i, i - n] += 1
     with np.errstate(divide="ignore"):
         return np.log(cnt)
+
+
+def prior_bias(beta, *, window, dists, sinks=0):
+    """[..., T, T] bias log(c_local_ij + c_offset_ij * exp(beta_i)) for
+    beta [..., T]: local = window and sinks, offset = integer distances
+    (duplicates counted); -inf where key j is not attended."""
+    beta = np.asarray(beta, dtype=np.float64)
+    T = beta.shape[-1]
+    loc = np.zeros((T, T))
+    off = np.zeros((T, T))
+    for i in range(T):
+        for t in range(window):
+            if i - t >= 0:
+                loc[i, i - t] += 1
+        for j in range(sinks):
+            if j <= i:
+                loc[i, j] += 1
+        for n in dists:
+            if i - n >= 0:
+                off[i, i - n] += 1
+    w = loc + off * np.exp(beta)[..., :, None]
+    with np.errstate(divide="ignore"):
+        return np.log(w)

@@ -12,7 +12,7 @@ import os
 
 import numpy as np
 
-from independent import dense_causal, integer_gather, multiset_bias, rope_complex
+from independent import dense_causal, integer_gather, multiset_bias, prior_bias, rope_complex
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
@@ -337,7 +337,91 @@ def pin_decode_dense_and_gather(orc):
             _close(lse, lf[..., pos], 1e-12, what=f"decode vs forward LSE alpha={alpha}")
 
 
+# -- log-prior on the offset members (pi-Attention's fusion in one softmax) ---
+
+def pin_log_prior_dense(orc):
+    """Integer distances with a per-query log-prior beta on the offset members:
+    dense causal attention whose bias gives key j of query i the weight
+    (local multiplicity) + (offset multiplicity) * e^beta_i."""
+    T = 60
+    q, k, v = (_rand((1, 1, 2, T, 8), s) for s in (130, 131, 132))
+    beta = 1.5 * _rand((1, 1, 2, T), 133)
+    for alpha, window, sinks in ((1.0, 4, 2), (2.0, 3, 0)):
+        dists = [int(alpha) * f for f in FIB]
+        o, lse = orc.fwd(q, k, v, [alpha], window=window, sinks=sinks, beta=beta)
+        bias = prior_bias(beta, window=window, dists=dists, sinks=sinks)
+        o_ref, lse_ref = dense_causal(q, k, v, bias=bias)
+        _close(o, o_ref, 1e-12, what=f"log-prior O alpha={alpha}")
+        _close(lse, lse_ref, 1e-12, what=f"log-prior LSE alpha={alpha}")
+
+
+def pin_log_prior_limits(orc):
+    """beta = ln 2 counts every offset member twice (the offset list given
+    twice, duplicates kept); beta = -800 (e^beta = 0 in fp64) removes the
+    offsets: forward and backward equal the oracle without offsets, and dbeta
+    is 0.  Interpolated alphas."""
+    q, k, v, do = (_rand((2, 1, 1, 45, 8), s) for s in (140, 141, 142, 143))
+    alpha = np.float32([0.73, 1.41])
+    kw = dict(window=4, sinks=1)
+    ln2 = np.full((2, 1, 1, 45), np.log(2.0))
+    o, lse = orc.fwd(q, k, v, alpha, beta=ln2, **kw)
+    o2, lse2 = orc.fwd(q, k, v, alpha, offsets=FIB + FIB, **kw)
+    _close(o, o2, 1e-12, what="beta = ln 2 vs doubled offsets, O")
+    _close(lse, lse2, 1e-12, what="beta = ln 2 vs doubled offsets, LSE")
+    g = orc.bwd(q, k, v, do, alpha, beta=ln2, **kw)
+    g2 = orc.bwd(q, k, v, do, alpha, offsets=FIB + FIB, **kw)
+    for name, a, b in zip(("dQ", "dK", "dV", "dalpha"), g[:4], g2):
+        _close(a, b, 1e-11, 1e-11, what=f"beta = ln 2 vs doubled offsets, {name}")
+    off = np.full((2, 1, 1, 45), -800.0)
+    o, lse = orc.fwd(q, k, v, alpha, beta=off, **kw)
+    o0, lse0 = orc.fwd(q, k, v, alpha, offsets=(), **kw)
+    _close(o, o0, 1e-12, what="beta = -800 vs no offsets, O")
+    _close(lse, lse0, 1e-12, what="beta = -800 vs no offsets, LSE")
+    g = orc.bwd(q, k, v, do, alpha, beta=off, **kw)
+    g0 = orc.bwd(q, k, v, do, alpha, offsets=(), **kw)
+    for name, a, b in zip(("dQ", "dK", "dV", "dalpha"), g[:4], g0):
+        _close(a, b, 1e-12, what=f"beta = -800 vs no offsets, {name}")
+    assert np.all(g[4] == 0.0), "dbeta with vanishing offset weights"
+
+
+def pin_fd_beta(orc):
+    """Central finite differences of sum(dO * O) for dbeta and, with the prior
+    present, for dQ, dK, dV and dalpha (interpolated alphas)."""
+    q, k, v, do = _fd_problem()
+    beta = 0.8 * _rand((2, 1, 2, 40), 150)
+    dq, dk, dv, dal, dbeta = orc.bwd(q, k, v, do, FD_ALPHA, beta=beta, **FD_KW)
+
+    def loss(qq, kk, vv, bb, al=FD_ALPHA):
+        return float((orc.fwd(qq, kk, vv, al, beta=bb, **FD_KW)[0] * do).sum())
+
+    h = 1e-6
+    rng = np.random.default_rng(6)
+    idxs = [tuple(rng.integers(0, s) for s in beta.shape) for _ in range(40)]
+    idxs += [(0, 0, 0, 0), (1, 0, 1, 39), (0, 0, 1, 2)]
+    for idx in idxs:
+        bp, bm = beta.copy(), beta.copy()
+        bp[idx] += h
+        bm[idx] -= h
+        fd = (loss(q, k, v, bp) - loss(q, k, v, bm)) / (2 * h)
+        assert abs(fd - dbeta[idx]) <= 1e-6 + 1e-6 * abs(fd), ("dbeta", idx, fd, dbeta[idx])
+    for name, grad, which in (("dQ", dq, 0), ("dK", dk, 1), ("dV", dv, 2)):
+        for idx in [tuple(rng.integers(0, s) for s in q.shape) for _ in range(20)]:
+            args_p = [q.copy(), k.copy(), v.copy()]
+            args_m = [q.copy(), k.copy(), v.copy()]
+            args_p[which][idx] += h
+            args_m[which][idx] -= h
+            fd = (loss(*args_p, beta) - loss(*args_m, beta)) / (2 * h)
+            assert abs(fd - grad[idx]) <= 1e-6 + 1e-6 * abs(fd), (name, idx, fd, grad[idx])
+    for l in range(2):
+        ap, am = FD_ALPHA.copy(), FD_ALPHA.copy()
+        ap[l] = np.float32(FD_ALPHA[l] + 3e-4)
+        am[l] = np.float32(FD_ALPHA[l] - 3e-4)
+        fd = (loss(q, k, v, beta, ap) - loss(q, k, v, beta, am)) / (float(ap[l]) - float(am[l]))
+        assert abs(fd - dal[l]) <= 2e-3 * abs(fd) + 1e-6, ("dalpha", l, fd, dal[l])
+
+
 ALL_PINS = [pin_geometry, pin_rope, pin_dense_limit, pin_integer_gather, pin_multiset,
             pin_softmax, pin_constant_v, pin_interp_continuity, pin_nan_geometry,
             pin_fp32_build, pin_fd_inputs, pin_fd_alpha, pin_theta_map,
-            pin_decode_dense_and_gather]
+            pin_decode_dense_and_gather, pin_log_prior_dense, pin_log_prior_limits,
+            pin_fd_beta]

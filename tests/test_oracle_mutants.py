@@ -40,6 +40,16 @@ MUTANTS = [
     ("decode_key_position", "rope_row(Ku + mb[m].a * D, mb[m].a, D, rope_base, ka);",
      "rope_row(Ku + mb[m].a * D, pos, D, rope_base, ka);"),
     ("decode_second_key_weight", "v += mb[m].wb * dot(qh, kb, D);", "v += mb[m].wa * dot(qh, kb, D);"),
+    ("prior_on_window", "sc[m] = dot(qh, row, D);\n        if (beta && mb[m].kind == 2)",
+     "sc[m] = dot(qh, row, D);\n        if (beta && mb[m].kind != 1)"),
+    ("prior_sign", "sc[m] = dot(qh, row, D);\n        if (beta && mb[m].kind == 2) sc[m] += beta",
+     "sc[m] = dot(qh, row, D);\n        if (beta && mb[m].kind == 2) sc[m] -= beta"),
+    ("prior_key_index", "sc[m] = dot(qh, row, D);\n        if (beta && mb[m].kind == 2) sc[m] += beta[u * T + i];",
+     "sc[m] = dot(qh, row, D);\n        if (beta && mb[m].kind == 2) sc[m] += beta[u * T + mb[m].a];"),
+    ("bwd_prior_missing", "sc[m] = dot(qh, krow + m * D, D);\n        if (beta && mb[m].kind == 2)",
+     "sc[m] = dot(qh, krow + m * D, D);\n        if (beta && mb[m].kind == 99)"),
+    ("dbeta_all_members", "if (mb[m].kind == 2) dbet += gs;", "dbet += gs;"),
+    ("dbeta_uses_p", "if (mb[m].kind == 2) dbet += gs;", "if (mb[m].kind == 2) dbet += pm;"),
     ("decode_query_scale", "for (int d = 0; d < D; ++d) qh[d] = (real)s * qh[d];\n    int n = members_of(pos",
      "for (int d = 0; d < D; ++d) qh[d] = qh[d];\n    int n = members_of(pos"),
 ]
