@@ -36,15 +36,17 @@ FALLBACK_HBM_GBS = 6650.0
 #   bwd key  : read Q, K, V, dO, LSE, D; write dK, dV
 #   RoPE pre-pass (rope_keys / rope_queries): read K (or Q), write it rotated
 # (the whole backward: Q, K, V, O, dO, dQ, dK, dV and LSE = 1028 B)
-def alg_bytes_per_token_head(kernel, D, elt, context=0):
+def alg_bytes_per_token_head(kernel, D, elt, context=0, prior=False):
     """Bytes a kernel must move per token-head: every input row read once and
     every output written once.  ``context``: bytes per token-head the saving
-    forward also writes into the training context (0 without one)."""
+    forward also writes into the training context (0 without one); ``prior``:
+    the fp32 log-prior is read by the forward and the query side, which also
+    writes its gradient."""
     row = D * elt
     if kernel.startswith("fwd"):
-        return 4 * row + 4 + context
+        return 4 * row + 4 + context + (4 if prior else 0)
     if kernel.startswith("bwd_q"):
-        return 6 * row + 8
+        return 6 * row + 8 + (8 if prior else 0)
     if kernel.startswith("bwd_kv"):
         return 6 * row + 8
     if kernel.startswith("rope"):      # RoPE pre-pass: read a row, write it rotated
@@ -200,10 +202,14 @@ def oracle_sample(wl, budget_s):
     def one_layer(l):
         ts = make_inputs(wl, layers=range(l, l + 1))
         arr = [t.float().numpy() for t in ts]
+        pkw = dict(kw)
+        if wl.prior:
+            from structured_sparse_attention_fibonacci_b200.inputs import make_prior
+            pkw["beta"] = make_prior(wl, layers=range(l, l + 1)).numpy()
         t0 = time.perf_counter()
-        oracle.fwd(arr[0], arr[1], arr[2], alpha[l:l + 1], **kw)
+        oracle.fwd(arr[0], arr[1], arr[2], alpha[l:l + 1], **pkw)
         if wl.backward:
-            oracle.bwd(arr[0], arr[1], arr[2], arr[3], alpha[l:l + 1], **kw)
+            oracle.bwd(arr[0], arr[1], arr[2], arr[3], alpha[l:l + 1], **pkw)
         return time.perf_counter() - t0
 
     t = one_layer(0)
@@ -255,6 +261,8 @@ def workload_config(wl, world):
                                                                   144, 233, 377, 610, 987)
                         else list(wl.offsets)),
             "alpha": wl.alpha_kind, "pass": pass_,
+            **({"prior": "log-prior beta ~ N(0, 1) per query on the offset members"}
+               if wl.prior else {}),
             "global_batch": wl.B * world, "seq_len": wl.T, "parallelism": f"replicas{world}",
             "l2": ("inputs larger than L2 (no flush needed)" if not wl.decode else
                    "KV caches (1 GiB) larger than L2; each step gathers 42 rows per unit")}
@@ -271,8 +279,13 @@ def run_ours(args, rank, world, local_rank):
     wl = WORKLOADS[args.workload]
     wl_rank = wl.shrink(seed=wl.seed + 100000 * rank) if world > 1 else wl
     host = make_inputs(wl_rank, pin=True)
+    if wl.prior:
+        from structured_sparse_attention_fibonacci_b200.inputs import make_prior
+        host = host + (make_prior(wl_rank, pin=True),)
     q, k, v = (t.to(dev) for t in host[:3])
     do = host[3].to(dev) if wl.backward else None
+    beta = host[-1].to(dev) if wl.prior else None
+    dbeta = torch.empty_like(beta) if wl.prior and wl.backward else None
     alpha_h = wl.alpha().pin_memory()
     alpha = alpha_h.to(dev)
     kw = dict(window=wl.window, sinks=wl.sinks, offsets=wl.offsets, rope_base=wl.rope_base)
@@ -290,11 +303,12 @@ def run_ours(args, rank, world, local_rank):
     launches = [0]
 
     def step():
-        sa.fwd(q, k, v, alpha, out=o, lse=lse, context=ctx if wl.backward else None, **kw)
+        sa.fwd(q, k, v, alpha, out=o, lse=lse, context=ctx if wl.backward else None, beta=beta,
+               **kw)
         n = sa.last_launch_count()
         if wl.backward:
             sa.bwd(q, k, v, o, lse, do, alpha, dq=dq, dk=dk, dv=dv, dalpha=dal, workspace=ws,
-                   context=ctx, **kw)
+                   context=ctx, beta=beta, dbeta=dbeta, **kw)
             n += sa.last_launch_count()
         launches[0] += n
 
@@ -346,7 +360,7 @@ def run_ours(args, rank, world, local_rank):
     # the training context per token-head: fp32 probabilities of every
     # member, fp32 row-score differences per offset, the fp16 rotated query
     ctx_th = ((wl.window + wl.sinks + 2 * len(wl.offsets)) * 4 + wl.D * 2) if wl.backward else 0
-    per_th = alg_bytes_per_token_head(dominant, wl.D, elt, ctx_th)
+    per_th = alg_bytes_per_token_head(dominant, wl.D, elt, ctx_th, wl.prior)
     bytes_launch = per_th * wl.token_heads
     achieved = bytes_launch / (kernels[dominant]["ms_per_launch"] / 1e3) / 1e9
     key = f"{wl.name}/{dominant}@{kernel_source_hash()}"
@@ -356,7 +370,7 @@ def run_ours(args, rank, world, local_rank):
                 "alg_bytes_per_launch": bytes_launch,
                 "traffic": traffic * wl.token_heads if traffic is not None else None}
     for n, kk in kernels.items():
-        b = alg_bytes_per_token_head(n, wl.D, elt, ctx_th) * wl.token_heads
+        b = alg_bytes_per_token_head(n, wl.D, elt, ctx_th, wl.prior) * wl.token_heads
         kk["alg_GBps"] = b / (kk["ms_per_launch"] / 1e3) / 1e9 if b else None
 
     # End to end through the public API: every step copies its inputs in from
@@ -364,7 +378,8 @@ def run_ours(args, rank, world, local_rank):
     # and three streams (copy in, compute, copy out) let step n's results
     # travel to the host while step n+1's inputs arrive and step n+1 runs;
     # a set is refilled only after its previous results have left.
-    h_in = [t for t in host[:3]] + ([host[3]] if wl.backward else [])
+    h_in = [t for t in host[:3]] + ([host[3]] if wl.backward else []) + \
+        ([host[-1]] if wl.prior else [])
     h2d = sum(t.numel() * t.element_size() for t in h_in) + alpha_h.numel() * 4
     sets = []
     for b in range(2):
@@ -374,6 +389,8 @@ def run_ours(args, rank, world, local_rank):
         if wl.backward:
             d_out += [torch.empty_like(q), torch.empty_like(q), torch.empty_like(q),
                       torch.empty(wl.L, dtype=torch.float32, device=dev)]
+            if wl.prior:
+                d_out += [torch.empty_like(beta)]
         h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d_out]
         sets.append((d_in, d_alpha, d_out, h_out))
     d2h = sum(t.numel() * t.element_size() for t in sets[0][2])
@@ -395,16 +412,15 @@ def run_ours(args, rank, world, local_rank):
             ev_in[b].record(s_in)
         with torch.cuda.stream(s_run):
             s_run.wait_event(ev_in[b])
-            if wl.backward:
-                qq, kk_, vv, dd = d_in
-            else:
-                (qq, kk_, vv), dd = d_in, None
+            qq, kk_, vv = d_in[:3]
+            dd = d_in[3] if wl.backward else None
+            bb = d_in[-1] if wl.prior else None
             sa.fwd(qq, kk_, vv, d_alpha, out=d_out[0], lse=d_out[1], stream=s_run,
-                   context=ctx if wl.backward else None, **kw)
+                   context=ctx if wl.backward else None, beta=bb, **kw)
             if wl.backward:
                 sa.bwd(qq, kk_, vv, d_out[0], d_out[1], dd, d_alpha, dq=d_out[2], dk=d_out[3],
                        dv=d_out[4], dalpha=d_out[5], workspace=ws, stream=s_run, context=ctx,
-                       **kw)
+                       beta=bb, dbeta=d_out[6] if wl.prior else None, **kw)
             ev_run[b].record(s_run)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_run[b])

@@ -166,6 +166,41 @@ sa_status sparse_attn_bwd_ctx(const sa_params* p, const void* q, const void* k, 
                               void* stream);
 
 /*
+ * Log-prior on the offset members.  "pi-Attention: Periodic Sparse
+ * Transformers for Efficient Long-Context Modeling" (Core components, dynamic
+ * adaptive fusion) merges its local and skip logits into one softmax by adding
+ * a log-prior in the log domain.  A softmax ignores a shift common to all of a
+ * query's members, so only the difference of the two priors matters.  Here
+ * one value beta_i per query is added to the score of every offset member of
+ * query i.  The window and the sinks get 0.  beta_i = ln 2 weighs each offset
+ * member as if it were listed twice; beta_i -> -inf removes the offsets.
+ *   beta  : device fp32 [L][B][H][T]                              (read)
+ *   dbeta : device fp32 [L][B][H][T], overwritten with
+ *           dLoss/dbeta_i = sum over query i's offset members of dLoss/dscore
+ *                                                                 (written)
+ * sparse_attn_fwd_prior: arguments as sparse_attn_fwd plus beta. context
+ *   NULL runs the plain forward. The bf16 / D = 64 configurations then use
+ *   the CUDA-core staged kernel whatever sparse_attn_select_forward says:
+ *   the tensor-core forward has no prior. A non-NULL context runs the training
+ *   forward (as sparse_attn_fwd_train): the saved probabilities include the
+ *   prior, and workspace is unused.
+ * sparse_attn_bwd_prior: arguments as sparse_attn_bwd plus beta (the
+ *   forward's), an optional context (from sparse_attn_fwd_prior with the same
+ *   beta; lse may then be NULL) and dbeta.
+ * beta, dbeta: non-NULL, 4-byte aligned, else SA_ERR_INVALID_ARG.  Decode and
+ * the allocation-free forward take no prior.
+ */
+sa_status sparse_attn_fwd_prior(const sa_params* p, const void* q, const void* k, const void* v,
+                                const float* alpha, const float* beta, void* o, float* lse,
+                                void* workspace, size_t workspace_bytes, void* context,
+                                size_t context_bytes, void* stream);
+sa_status sparse_attn_bwd_prior(const sa_params* p, const void* q, const void* k, const void* v,
+                                const void* o, const float* lse, const void* dout,
+                                const float* alpha, const float* beta, const void* context,
+                                void* dq, void* dk, void* dv, float* dalpha, float* dbeta,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Single-token decode with a KV cache: for every (layer, batch, head), the
  * attention output of one new query at position `pos` against the cache rows
  * 0..pos (the new token's own K/V row, at pos, included).  The result equals

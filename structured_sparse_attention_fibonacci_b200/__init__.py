@@ -34,7 +34,8 @@ EXPORTED = ("sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_workspace_size",
             "sparse_attn_trace_enable", "sparse_attn_trace_read", "sparse_attn_force_general",
             "sparse_attn_fwd_noalloc", "sparse_attn_device_error", "sparse_attn_select_forward",
             "sparse_attn_context_size", "sparse_attn_fwd_train", "sparse_attn_bwd_ctx",
-            "sparse_attn_decode", "sparse_attn_alpha_from_theta", "sparse_attn_dtheta")
+            "sparse_attn_decode", "sparse_attn_alpha_from_theta", "sparse_attn_dtheta",
+            "sparse_attn_fwd_prior", "sparse_attn_bwd_prior")
 
 
 class SaParams(ctypes.Structure):
@@ -93,6 +94,12 @@ def lib():
         L.sparse_attn_bwd_ctx.restype = ctypes.c_int
         L.sparse_attn_bwd_ctx.argtypes = [P, vp, vp, vp, vp, fp, vp, fp, vp, vp, vp, vp, fp, vp,
                                           ctypes.c_size_t, vp]
+        L.sparse_attn_fwd_prior.restype = ctypes.c_int
+        L.sparse_attn_fwd_prior.argtypes = [P, vp, vp, vp, fp, fp, vp, fp, vp, ctypes.c_size_t,
+                                            vp, ctypes.c_size_t, vp]
+        L.sparse_attn_bwd_prior.restype = ctypes.c_int
+        L.sparse_attn_bwd_prior.argtypes = [P, vp, vp, vp, vp, fp, vp, fp, fp, vp, vp, vp, vp, fp,
+                                            fp, vp, ctypes.c_size_t, vp]
         L.sparse_attn_select_forward.restype = None
         L.sparse_attn_select_forward.argtypes = [ctypes.c_int]
         L.sparse_attn_device_error.restype = ctypes.c_int32
@@ -203,15 +210,29 @@ def context_size(shape, dtype, **kw) -> int:
     return int(lib().sparse_attn_context_size(ctypes.byref(p)))
 
 
+def _check_prior(shape, dev, **named):
+    for name, t in named.items():
+        if (t.device != dev or not t.is_contiguous() or t.dtype != torch.float32
+                or tuple(t.shape) != tuple(shape[:4])):
+            raise ValueError(f"{name} must be a contiguous CUDA fp32 tensor of shape "
+                             f"{tuple(shape[:4])}")
+
+
 def fwd(q, k, v, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0, scale=0.0,
-        out=None, lse=None, want_lse=True, stream=None, context=None):
+        out=None, lse=None, want_lse=True, stream=None, context=None, beta=None):
     """Sparse attention forward over all layers: returns (O, LSE or None).
 
     q, k, v: CUDA tensors [L, B, H, T, D] (bf16 or fp32, contiguous).
     alpha: CUDA fp32 [L].  Output buffers may be passed in via out= / lse=.
     context: a CUDA uint8 buffer of context_size() bytes: the forward then
     runs as sparse_attn_fwd_train and saves what bwd(..., context=) reuses.
+    beta: CUDA fp32 [L, B, H, T], a log-prior added to every offset member's
+    score of each query (sparse_attn_fwd_prior).
     """
+    if beta is not None:
+        return _fwd_prior(q, k, v, alpha, beta, window=window, offsets=offsets, sinks=sinks,
+                          rope_base=rope_base, scale=scale, out=out, lse=lse, want_lse=want_lse,
+                          stream=stream, context=context)
     if context is not None:
         return _fwd_train(q, k, v, alpha, window=window, offsets=offsets, sinks=sinks,
                           rope_base=rope_base, scale=scale, out=out, lse=lse, want_lse=want_lse,
@@ -229,6 +250,27 @@ def fwd(q, k, v, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0, sc
     st = L.sparse_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(out),
                            _ptr(lse), _ptr(ws), ws_n, _stream_handle(stream))
     _check("sparse_attn_fwd", st)
+    return out, lse
+
+
+def _fwd_prior(q, k, v, alpha, beta, *, window, offsets, sinks, rope_base, scale, out, lse,
+               want_lse, stream, context):
+    shape, dtype, dev = tuple(q.shape), q.dtype, q.device
+    if lse is None and want_lse:
+        lse = torch.empty(shape[:4], dtype=torch.float32, device=dev)
+    out = torch.empty_like(q) if out is None else out
+    _check_tensors(shape, dtype, dev, q=q, k=k, v=v, o=out, alpha=alpha, lse=lse)
+    _check_prior(shape, dev, beta=beta)
+    p = make_params(shape, dtype, window=window, offsets=offsets, sinks=sinks,
+                    rope_base=rope_base, scale=scale)
+    L = lib()
+    ws_n = int(L.sparse_attn_workspace_size(ctypes.byref(p), 0)) if context is None else 0
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=dev) if ws_n else None
+    st = L.sparse_attn_fwd_prior(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                 _ptr(beta), _ptr(out), _ptr(lse), _ptr(ws), ws_n, _ptr(context),
+                                 context.numel() if context is not None else 0,
+                                 _stream_handle(stream))
+    _check("sparse_attn_fwd_prior", st)
     return out, lse
 
 
@@ -321,11 +363,13 @@ def fwd_noalloc(q, k, v, alpha, *, window, offsets=FIB15, sinks=0, rope_base=100
 
 def bwd(q, k, v, o, lse, dout, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0,
         scale=0.0, dq=None, dk=None, dv=None, dalpha=None, workspace=None, stream=None,
-        context=None):
+        context=None, beta=None, dbeta=None):
     """Sparse attention backward: returns (dQ, dK, dV, dalpha[L]).
 
     context: the buffer a fwd(..., context=) call filled for the same inputs;
-    the backward then runs as sparse_attn_bwd_ctx (no score pass)."""
+    the backward then runs as sparse_attn_bwd_ctx (no score pass).
+    beta: the forward's log-prior [L, B, H, T]; the call then runs as
+    sparse_attn_bwd_prior and returns (dQ, dK, dV, dalpha, dbeta)."""
     shape, dtype, dev = tuple(q.shape), q.dtype, q.device
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
@@ -339,6 +383,16 @@ def bwd(q, k, v, o, lse, dout, alpha, *, window, offsets=FIB15, sinks=0, rope_ba
     ws_n = int(L.sparse_attn_workspace_size(ctypes.byref(p), 1))
     if workspace is None or workspace.numel() < ws_n:
         workspace = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev)
+    if beta is not None:
+        dbeta = torch.empty(shape[:4], dtype=torch.float32, device=dev) if dbeta is None else dbeta
+        _check_prior(shape, dev, beta=beta, dbeta=dbeta)
+        st = L.sparse_attn_bwd_prior(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                     _ptr(lse), _ptr(dout), _ptr(alpha), _ptr(beta),
+                                     _ptr(context), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dalpha),
+                                     _ptr(dbeta), _ptr(workspace), workspace.numel(),
+                                     _stream_handle(stream))
+        _check("sparse_attn_bwd_prior", st)
+        return dq, dk, dv, dalpha, dbeta
     if context is not None:
         st = L.sparse_attn_bwd_ctx(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                                    _ptr(dout), _ptr(alpha), _ptr(context), _ptr(dq), _ptr(dk),

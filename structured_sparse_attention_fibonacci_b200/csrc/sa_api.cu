@@ -202,15 +202,20 @@ size_t sparse_attn_workspace_size(const sa_params* p, int backward) {
   return need;
 }
 
-sa_status sparse_attn_fwd(const sa_params* p, const void* q, const void* k, const void* v,
-                          const float* alpha, void* o, float* lse, void* workspace,
-                          size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared by sparse_attn_fwd and sparse_attn_fwd_prior (beta may be null).
+sa_status fwd_impl(const sa_params* p, const void* q, const void* k, const void* v,
+                   const float* alpha, const float* beta, void* o, float* lse, void* workspace,
+                   size_t workspace_bytes, void* stream) {
   sa::Problem pb;
   sa_status s = build_problem(p, &pb);
   if (s != SA_OK) return s;
   if (!q || !k || !v || !alpha || !o) return SA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (lse && !aligned4(lse)) || !aligned4(alpha))
+      (lse && !aligned4(lse)) || !aligned4(alpha) || (beta && !aligned4(beta)))
     return SA_ERR_INVALID_ARG;
   const size_t need = sparse_attn_workspace_size(p, 0);
   if (workspace_bytes < need || (need && (!workspace || !aligned16(workspace))))
@@ -218,19 +223,125 @@ sa_status sparse_attn_fwd(const sa_params* p, const void* q, const void* k, cons
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const float2* rope = nullptr;
   if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
-  sa::FwdPtrs a = {q, k, v, alpha, o, lse, rope};
+  sa::FwdPtrs a = {q, k, v, alpha, o, lse, rope, beta};
   int launches = 0;
   cudaError_t e;
   if (g_force_general || !sa::fast_fwd_supported(pb))
     e = sa::launch_fwd_general(pb, a, st, &launches);
-  else if (g_fwd_select == 2 ? sa::tc_fwd_supported(pb)
-                              : (g_fwd_select == 0 && sa::tc_fwd_preferred(pb)))
-    e = sa::launch_fwd_tc(pb, a, workspace, st, &launches);
+  else if (!beta && (g_fwd_select == 2 ? sa::tc_fwd_supported(pb)
+                                       : (g_fwd_select == 0 && sa::tc_fwd_preferred(pb))))
+    e = sa::launch_fwd_tc(pb, a, workspace, st, &launches);   // (no log-prior there)
   else
     e = sa::launch_fwd_fast(pb, a, workspace, st, &launches);
   if (e != cudaSuccess) return SA_ERR_CUDA;
   g_last_launches = launches;
   return SA_OK;
+}
+
+// Shared by sparse_attn_fwd_train and sparse_attn_fwd_prior with a context.
+sa_status fwd_train_impl(const sa_params* p, const void* q, const void* k, const void* v,
+                         const float* alpha, const float* beta, void* o, float* lse,
+                         void* context, size_t context_bytes, void* stream) {
+  sa::Problem pb;
+  sa_status s = build_problem(p, &pb);
+  if (s != SA_OK) return s;
+  if (!q || !k || !v || !alpha || !o) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse && !aligned4(lse)) || !aligned4(alpha) || (beta && !aligned4(beta)))
+    return SA_ERR_INVALID_ARG;
+  const size_t need = sparse_attn_context_size(p);
+  if (need == 0) return SA_ERR_UNSUPPORTED;
+  if (context_bytes < need || !context || !aligned16(context)) return SA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float2* rope = nullptr;
+  if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
+  sa::FwdPtrs a = {q, k, v, alpha, o, lse, rope, beta};
+  const sa::CtxLayout cl = sa::ctx_layout(pb);
+  char* cb = reinterpret_cast<char*>(context);
+  int launches = 0;
+  if (sa::launch_fwd_fast(pb, a, cb + cl.khat_off, st, &launches,
+                          reinterpret_cast<float*>(cb + cl.p_off),
+                          reinterpret_cast<float*>(cb + cl.dt_off), cb + cl.qhat_off) !=
+      cudaSuccess)
+    return SA_ERR_CUDA;
+  g_last_launches = launches;
+  return SA_OK;
+}
+
+// Shared by sparse_attn_bwd, sparse_attn_bwd_ctx and sparse_attn_bwd_prior
+// (beta / dbeta may be null; a context selects the context backward).
+sa_status bwd_impl(const sa_params* p, const void* q, const void* k, const void* v,
+                   const void* o, const float* lse, const void* dout, const float* alpha,
+                   const float* beta, const void* context, void* dq, void* dk, void* dv,
+                   float* dalpha, float* dbeta, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  sa::Problem pb;
+  sa_status s = build_problem(p, &pb);
+  if (s != SA_OK) return s;
+  const void* tensors[] = {q, k, v, o, dout, dq, dk, dv};
+  for (const void* x : tensors)
+    if (!x || !aligned16(x)) return SA_ERR_INVALID_ARG;
+  const void* vectors[] = {alpha, dalpha};
+  for (const void* x : vectors)
+    if (!x || !aligned4(x)) return SA_ERR_INVALID_ARG;
+  if ((lse && !aligned4(lse)) || (beta && !aligned4(beta)) || (dbeta && !aligned4(dbeta)))
+    return SA_ERR_INVALID_ARG;
+  size_t need;
+  if (context) {
+    if (sparse_attn_context_size(p) == 0) return SA_ERR_UNSUPPORTED;
+    if (!aligned16(context)) return SA_ERR_INVALID_ARG;
+    need = sa::fast_bwd_workspace(pb);
+    if (workspace_bytes < need || !workspace || !aligned16(workspace)) return SA_ERR_WORKSPACE;
+  } else {
+    if (!lse) return SA_ERR_INVALID_ARG;
+    need = sparse_attn_workspace_size(p, 1);
+    if (workspace_bytes < need || (need && (!workspace || !aligned16(workspace))))
+      return SA_ERR_WORKSPACE;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float2* rope = nullptr;
+  if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
+  sa::BwdPtrs a = {q, k, v, o, dout, lse, alpha, dq, dk, dv, dalpha, rope, workspace, beta, dbeta};
+  int launches = 0;
+  cudaError_t e;
+  if (context)
+    e = sa::launch_bwd_fast(pb, a, st, &launches, context);
+  else
+    e = (!g_force_general && sa::fast_bwd_supported(pb))
+            ? sa::launch_bwd_fast(pb, a, st, &launches)
+            : sa::launch_bwd_general(pb, a, st, &launches);
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+  g_last_launches = launches;
+  return SA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sa_status sparse_attn_fwd(const sa_params* p, const void* q, const void* k, const void* v,
+                          const float* alpha, void* o, float* lse, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  return fwd_impl(p, q, k, v, alpha, nullptr, o, lse, workspace, workspace_bytes, stream);
+}
+
+sa_status sparse_attn_fwd_prior(const sa_params* p, const void* q, const void* k, const void* v,
+                                const float* alpha, const float* beta, void* o, float* lse,
+                                void* workspace, size_t workspace_bytes, void* context,
+                                size_t context_bytes, void* stream) {
+  if (!beta) return SA_ERR_INVALID_ARG;
+  return context ? fwd_train_impl(p, q, k, v, alpha, beta, o, lse, context, context_bytes, stream)
+                 : fwd_impl(p, q, k, v, alpha, beta, o, lse, workspace, workspace_bytes, stream);
+}
+
+sa_status sparse_attn_bwd_prior(const sa_params* p, const void* q, const void* k, const void* v,
+                                const void* o, const float* lse, const void* dout,
+                                const float* alpha, const float* beta, const void* context,
+                                void* dq, void* dk, void* dv, float* dalpha, float* dbeta,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!beta || !dbeta) return SA_ERR_INVALID_ARG;
+  return bwd_impl(p, q, k, v, o, lse, dout, alpha, beta, context, dq, dk, dv, dalpha, dbeta,
+                  workspace, workspace_bytes, stream);
 }
 
 sa_status sparse_attn_decode(const sa_params* p, int32_t pos, const void* q, const void* k,
@@ -286,30 +397,7 @@ size_t sparse_attn_context_size(const sa_params* p) {
 sa_status sparse_attn_fwd_train(const sa_params* p, const void* q, const void* k, const void* v,
                                 const float* alpha, void* o, float* lse, void* context,
                                 size_t context_bytes, void* stream) {
-  sa::Problem pb;
-  sa_status s = build_problem(p, &pb);
-  if (s != SA_OK) return s;
-  if (!q || !k || !v || !alpha || !o) return SA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (lse && !aligned4(lse)) || !aligned4(alpha))
-    return SA_ERR_INVALID_ARG;
-  const size_t need = sparse_attn_context_size(p);
-  if (need == 0) return SA_ERR_UNSUPPORTED;
-  if (context_bytes < need || !context || !aligned16(context)) return SA_ERR_WORKSPACE;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const float2* rope = nullptr;
-  if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
-  sa::FwdPtrs a = {q, k, v, alpha, o, lse, rope};
-  const sa::CtxLayout cl = sa::ctx_layout(pb);
-  char* cb = reinterpret_cast<char*>(context);
-  int launches = 0;
-  if (sa::launch_fwd_fast(pb, a, cb + cl.khat_off, st, &launches,
-                          reinterpret_cast<float*>(cb + cl.p_off),
-                          reinterpret_cast<float*>(cb + cl.dt_off), cb + cl.qhat_off) !=
-      cudaSuccess)
-    return SA_ERR_CUDA;
-  g_last_launches = launches;
-  return SA_OK;
+  return fwd_train_impl(p, q, k, v, alpha, nullptr, o, lse, context, context_bytes, stream);
 }
 
 sa_status sparse_attn_bwd_ctx(const sa_params* p, const void* q, const void* k, const void* v,
@@ -317,57 +405,18 @@ sa_status sparse_attn_bwd_ctx(const sa_params* p, const void* q, const void* k, 
                               const float* alpha, const void* context, void* dq, void* dk,
                               void* dv, float* dalpha, void* workspace, size_t workspace_bytes,
                               void* stream) {
-  sa::Problem pb;
-  sa_status s = build_problem(p, &pb);
-  if (s != SA_OK) return s;
-  const void* tensors[] = {q, k, v, o, dout, dq, dk, dv};
-  for (const void* x : tensors)
-    if (!x || !aligned16(x)) return SA_ERR_INVALID_ARG;
-  const void* vectors[] = {alpha, dalpha};
-  for (const void* x : vectors)
-    if (!x || !aligned4(x)) return SA_ERR_INVALID_ARG;
-  if (lse && !aligned4(lse)) return SA_ERR_INVALID_ARG;
-  if (sparse_attn_context_size(p) == 0) return SA_ERR_UNSUPPORTED;
-  if (!context || !aligned16(context)) return SA_ERR_INVALID_ARG;
-  const size_t need = sa::fast_bwd_workspace(pb);
-  if (workspace_bytes < need || !workspace || !aligned16(workspace)) return SA_ERR_WORKSPACE;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const float2* rope = nullptr;
-  if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
-  sa::BwdPtrs a = {q, k, v, o, dout, lse, alpha, dq, dk, dv, dalpha, rope, workspace};
-  int launches = 0;
-  if (sa::launch_bwd_fast(pb, a, st, &launches, context) != cudaSuccess) return SA_ERR_CUDA;
-  g_last_launches = launches;
-  return SA_OK;
+  if (!context) return SA_ERR_INVALID_ARG;
+  return bwd_impl(p, q, k, v, o, lse, dout, alpha, nullptr, context, dq, dk, dv, dalpha, nullptr,
+                  workspace, workspace_bytes, stream);
 }
 
 sa_status sparse_attn_bwd(const sa_params* p, const void* q, const void* k, const void* v,
                           const void* o, const float* lse, const void* dout, const float* alpha,
                           void* dq, void* dk, void* dv, float* dalpha, void* workspace,
                           size_t workspace_bytes, void* stream) {
-  sa::Problem pb;
-  sa_status s = build_problem(p, &pb);
-  if (s != SA_OK) return s;
-  const void* tensors[] = {q, k, v, o, dout, dq, dk, dv};
-  for (const void* x : tensors)
-    if (!x || !aligned16(x)) return SA_ERR_INVALID_ARG;
-  const void* vectors[] = {lse, alpha, dalpha};
-  for (const void* x : vectors)
-    if (!x || !aligned4(x)) return SA_ERR_INVALID_ARG;
-  const size_t need = sparse_attn_workspace_size(p, 1);
-  if (workspace_bytes < need || (need && (!workspace || !aligned16(workspace))))
-    return SA_ERR_WORKSPACE;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const float2* rope = nullptr;
-  if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
-  sa::BwdPtrs a = {q, k, v, o, dout, lse, alpha, dq, dk, dv, dalpha, rope, workspace};
-  int launches = 0;
-  cudaError_t e = (!g_force_general && sa::fast_bwd_supported(pb))
-                      ? sa::launch_bwd_fast(pb, a, st, &launches)
-                      : sa::launch_bwd_general(pb, a, st, &launches);
-  if (e != cudaSuccess) return SA_ERR_CUDA;
-  g_last_launches = launches;
-  return SA_OK;
+  if (!lse) return SA_ERR_INVALID_ARG;
+  return bwd_impl(p, q, k, v, o, lse, dout, alpha, nullptr, nullptr, dq, dk, dv, dalpha, nullptr,
+                  workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

@@ -48,6 +48,7 @@ struct FastArgs {
   float* save_p;                       // SAVE: [units][W+S+n_off][T] member probabilities
   float* save_dt;                      // SAVE: [units][n_off][T] row-score differences
   __half* save_q;                      // SAVE: [units][T][64] fp16 of RoPE(Q) * scale / 256
+  const float* beta;                   // log-prior on offset members [units][T], or nullptr
 };
 
 enum : int { kFar = 0, kNear = 1, kDead = 2 };
@@ -289,6 +290,8 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
 
   const int lr = 4 * gid + c;                  // this lane's query, tile-local
   const int i_own = ig + c;                    // ... and its position
+  // its log-prior on the offset members (0 without one)
+  const float prior = (a.beta && i_own < T) ? __ldg(a.beta + (size_t)unit * T + i_own) : 0.f;
   float mx = -INFINITY;                        // running max of its valid scores
   float* my_sc = sc + (size_t)lr * a.sc_stride;
   const int win_lo = i0 - W + 1, win_hi = i0 + M;
@@ -361,9 +364,10 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
         }
         float out[NV];
         reduce_scatter4<NV>(part, out, c);
-        my_sc[W + S + m] = out[0];
+        const float sv = out[0] + prior;
+        my_sc[W + S + m] = sv;
         if (SAVE && i_own < T) a.save_dt[((size_t)unit * n_off + m) * T + i_own] = out[NV - 1];
-        if (i_own - g.c >= 0) mx = fmaxf(mx, out[0]);
+        if (i_own - g.c >= 0) mx = fmaxf(mx, sv);
       }
       kk = nx;
     }
@@ -383,6 +387,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
         const OffGeo g = sg[kk];
         float sv = g.wa * my_sc[g.lo];
         if (g.w != 0.f) sv += g.w * my_sc[g.lo + 1];
+        sv += prior;
         my_sc[W + S + kk] = sv;
         if (SAVE)
           a.save_dt[((size_t)unit * n_off + kk) * T + i] = my_sc[g.lo + 1] - my_sc[g.lo];
@@ -544,6 +549,7 @@ cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& p, void* keys_ws, 
   a.alpha = p.alpha; a.rope = p.rope;
   a.o = reinterpret_cast<__nv_bfloat16*>(p.o); a.lse = p.lse;
   a.save_p = save_p; a.save_dt = save_dt; a.save_q = reinterpret_cast<__half*>(save_q);
+  a.beta = p.beta;
   cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&a.err), g_fwd_err);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((long long)pb.units() * a.n_tiles);

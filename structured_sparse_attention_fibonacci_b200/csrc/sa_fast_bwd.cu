@@ -54,6 +54,8 @@ struct FastBwdArgs {
   unsigned* err;
   const float* ctx_p;                    // training context: [units][W+S+n_off][T] probabilities
   const float* ctx_dt;                   // ... and [units][n_off][T] row-score differences
+  const float* beta;                     // log-prior on offset members [units][T], or nullptr
+  float* dbeta;                          // its gradient [units][T], or nullptr
 };
 
 enum : int { kFar = 0, kNear = 1, kDead = 2 };
@@ -178,7 +180,7 @@ __device__ __forceinline__ int member_dots(const FastBwdArgs& a, Stager& stg,
                                            const int* s_kind, int i0, int ig, int c, int off0,
                                            int d1, const float (&x)[4][16], float* val_row,
                                            float* diff_row, int i_own, float* mx,
-                                           const float* p_row, float* dal_u) {
+                                           const float* p_row, float* dal_u, float bias) {
   constexpr int M = kFastM;
   const int T = a.T, W = a.W, S = a.S, RB = a.ring_rows;
   const int win_lo = i0 - W + 1, win_hi = i0 + M;
@@ -244,6 +246,7 @@ __device__ __forceinline__ int member_dots(const FastBwdArgs& a, Stager& stg,
       }
       float out[2];
       reduce_scatter4<2>(part, out, c);
+      out[0] += bias;
       val_row[W + S + kk] = out[0];
       if (p_row) {
         if (i_own - g.lo - 1 >= 0)
@@ -310,6 +313,7 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
 #pragma unroll
         for (int h = 0; h < 8; ++h) x[h] = qnan;
         reinterpret_cast<uint4*>(a.dq + ub + (size_t)i * kD)[e % kChunks] = pack8(x);
+        if (e % kChunks == 0 && a.dbeta) a.dbeta[(size_t)unit * T + i] = qnan;
       }
     }
     if (t == 0) a.dal_part[(size_t)unit * a.n_tiles + tile] = qnan;
@@ -325,6 +329,8 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
   float x[4][16];
   const int i = ig + c;
   const int n_slot = W + S + n_off;
+  // this lane's query's log-prior on the offset members (0 without one)
+  const float prior = (!CTX && a.beta && i < T) ? __ldg(a.beta + (size_t)unit * T + i) : 0.f;
   float dal_v = 0.f, dal_u = 0.f;
   if (CTX) {
     // probabilities and row-score differences from the training context:
@@ -343,7 +349,7 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
     load_lane_rows<true>(Q, a.rope, ig, T, c, par, a.scale * kKeyUnstage, x);
     float mx = -INFINITY;   // running max of this lane's query's valid scores
     if (member_dots<true>(a, stg, ring, sinkb, Kh, sg, s_kind, i0, ig, c, off0, d1, x, my_sc,
-                          my_dt, ig + c, &mx, nullptr, nullptr))
+                          my_dt, ig + c, &mx, nullptr, nullptr, prior))
       return;
     // owner lane: probabilities from these scores (not the forward's LSE, so
     // that sum_m p_m = 1 and sum_m g_m = 0 hold for the values used here)
@@ -351,7 +357,7 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
       for (int kk = 0; kk < n_off; ++kk) {
         if (s_kind[kk] != kNear) continue;
         const OffGeo g = sg[kk];
-        my_sc[W + S + kk] = g.wa * my_sc[g.lo] + g.w * my_sc[g.lo + 1];
+        my_sc[W + S + kk] = g.wa * my_sc[g.lo] + g.w * my_sc[g.lo + 1] + prior;
         my_dt[kk] = my_sc[g.lo + 1] - my_sc[g.lo];
         if (i - g.c >= 0) mx = fmaxf(mx, my_sc[W + S + kk]);
       }
@@ -383,7 +389,7 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
   // pass 2: dO . values; far offsets add f_k p_k (dp_k dtau_k + dpi_k) to dal_u
   load_lane_rows<false>(dO, a.rope, ig, T, c, par, 1.f, x);
   if (member_dots<false>(a, stg, ring, sinkb, Vb, sg, s_kind, i0, ig, c, off0, d1, x, my_dp,
-                         my_dt, ig + c, nullptr, my_sc, &dal_u))
+                         my_dt, ig + c, nullptr, my_sc, &dal_u, 0.f))
     return;
   __syncthreads();
 
@@ -409,6 +415,11 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
         my_sc[m] = p != 0.f ? g : 0.f;      // p -> g (dsigma)
       }
       dal = dal_u - Dsum * dal_v;
+      if (a.dbeta) {                        // d log-prior: the offset members' g, summed
+        float db = 0.f;
+        for (int kk = 0; kk < n_off; ++kk) db += my_sc[W + S + kk];
+        a.dbeta[(size_t)unit * T + i] = db;
+      }
       for (int kk = 0; kk < n_off; ++kk) {  // fold near offsets into window weights
         if (s_kind[kk] != kNear) continue;
         const OffGeo g = sg[kk];
@@ -885,6 +896,7 @@ cudaError_t launch_bwd_fast(const Problem& pb, const BwdPtrs& p, cudaStream_t st
   a.dq = reinterpret_cast<__nv_bfloat16*>(p.dq);
   a.dk = reinterpret_cast<__nv_bfloat16*>(p.dk);
   a.dv = reinterpret_cast<__nv_bfloat16*>(p.dv);
+  a.beta = p.beta; a.dbeta = p.dbeta;
   char* ws = reinterpret_cast<char*>(p.workspace);
   const CtxLayout CL = ctx_layout(pb);
   const char* cb = reinterpret_cast<const char*>(ctx);

@@ -9,6 +9,11 @@
 // Capps), technical summary, Methodology -- "Attended set" (window plus
 // Fibonacci offsets), "Scaling" (d_k = alpha f_k), "Implementation" (linear
 // K/V interpolation so gradients reach alpha; RoPE before the gather).
+// Optional log-prior beta [units][T] on the offset members' scores
+// ("pi-Attention: Periodic Sparse Transformers for Efficient Long-Context
+// Modeling", Core components: local and skip logits fused in one softmax
+// through a log-prior), with its gradient dbeta = sum of the offset members'
+// dscores.
 #include "sa_device.cuh"
 #include "sa_internal.h"
 
@@ -28,6 +33,7 @@ struct GenArgs {
   float* dvec;                               // D_i = dO_i . O_i   [units][T]
   float* dal_part;                           // [units][n_tiles]
   float* sink_k; float* sink_v;              // [units][n_tiles][S][D]
+  const float* beta; float* dbeta;           // log-prior on offset members [units][T]
 };
 
 // Per-CTA offset geometry for this layer; returns nonzero when some offset
@@ -88,8 +94,9 @@ __global__ void __launch_bounds__(kGenWarps * 32) k_fwd_general(const GenArgs a)
   float m = -INFINITY, l = 0.f, o1[N], o2[N];
 #pragma unroll
   for (int h = 0; h < N; ++h) { o1[h] = 0.f; o2[h] = 0.f; }
+  const float prior = a.beta ? __ldg(a.beta + (size_t)unit * a.T + qi) : 0.f;
 
-  auto visit = [&](bool valid, int ra, int rb, float wa, float wb) {
+  auto visit = [&](bool valid, int ra, int rb, float wa, float wb, float bias) {
     float k1[N], k2[N];
     load_krot<T, D>(K, a.rope, valid ? ra : 0, j0, k1, k2);
     const bool two = valid && rb >= 0;
@@ -102,7 +109,7 @@ __global__ void __launch_bounds__(kGenWarps * 32) k_fwd_general(const GenArgs a)
     float part = 0.f;
 #pragma unroll
     for (int h = 0; h < N; ++h) part += q1[h] * k1[h] + q2[h] * k2[h];
-    const float s = group8_sum(part);
+    const float s = group8_sum(part) + bias;
     if (valid) {
       float v1[N], v2[N];
       load_plain<T, D>(V, ra, j0, v1, v2);
@@ -121,12 +128,12 @@ __global__ void __launch_bounds__(kGenWarps * 32) k_fwd_general(const GenArgs a)
     }
   };
 
-  for (int t = 0; t < a.W; ++t) visit(qi - t >= 0, qi - t, -1, 1.f, 0.f);
-  for (int s = 0; s < a.S; ++s) visit(s <= qi, s, -1, 1.f, 0.f);
+  for (int t = 0; t < a.W; ++t) visit(qi - t >= 0, qi - t, -1, 1.f, 0.f, 0.f);
+  for (int s = 0; s < a.S; ++s) visit(s <= qi, s, -1, 1.f, 0.f, 0.f);
   for (int k = 0; k < a.n_off; ++k) {
     const OffGeo g = sg[k];
     const int ra = qi - g.lo;
-    visit(g.ok && qi - g.c >= 0, ra, g.w != 0.f ? ra - 1 : -1, g.wa, g.w);
+    visit(g.ok && qi - g.c >= 0, ra, g.w != 0.f ? ra - 1 : -1, g.wa, g.w, prior);
   }
 
   if (active) {
@@ -181,10 +188,11 @@ __global__ void __launch_bounds__(kGenWarps * 32) k_bwd_q_general(const GenArgs 
     Dsum = group8_sum(part);
   }
   const float lse_i = __ldg(a.lse + (size_t)unit * a.T + qi);
+  const float prior = a.beta ? __ldg(a.beta + (size_t)unit * a.T + qi) : 0.f;
   float dq1[N], dq2[N];
 #pragma unroll
   for (int h = 0; h < N; ++h) { dq1[h] = 0.f; dq2[h] = 0.f; }
-  float dal = 0.f;
+  float dal = 0.f, dprior = 0.f;
 
   // One member: returns its dsigma (g) and p; both 0 when it does not exist.
   // koff >= 0 marks an offset member (adds its d-alpha term).
@@ -216,7 +224,7 @@ __global__ void __launch_bounds__(kGenWarps * 32) k_bwd_q_general(const GenArgs 
       s_part += q1[h] * key1[h] + q2[h] * key2[h];
       dp_part += g1[h] * v1 + g2[h] * v2;
     }
-    const float s = group8_sum(s_part);
+    const float s = group8_sum(s_part) + (koff >= 0 ? prior : 0.f);
     const float dp = group8_sum(dp_part);
     const float p = valid ? expf(s - lse_i) : 0.f;
     const float g = p * (dp - Dsum);
@@ -224,6 +232,7 @@ __global__ void __launch_bounds__(kGenWarps * 32) k_bwd_q_general(const GenArgs 
 #pragma unroll
       for (int h = 0; h < N; ++h) { dq1[h] += g * key1[h]; dq2[h] += g * key2[h]; }
     }
+    if (koff >= 0) dprior += g;
     if (has_b) {
       float t = 0.f;
 #pragma unroll
@@ -288,6 +297,7 @@ __global__ void __launch_bounds__(kGenWarps * 32) k_bwd_q_general(const GenArgs 
     store_row<T, N>(dQ + j0, dq1);
     store_row<T, N>(dQ + HALF + j0, dq2);
     if (c == 0) a.dvec[(size_t)unit * a.T + i] = Dsum;
+    if (c == 0 && a.dbeta) a.dbeta[(size_t)unit * a.T + i] = bad ? qnan : dprior;
   }
   // d-alpha partial of this CTA: butterfly over the warp, then warps in order.
 #pragma unroll
@@ -352,8 +362,9 @@ __global__ void __launch_bounds__(kGenWarps * 32) k_bwd_kv_general(const GenArgs
 #pragma unroll
   for (int h = 0; h < N; ++h) { dk1[h] = dk2[h] = dv1[h] = dv2[h] = 0.f; }
 
-  // Query i's member reads row r with weight wr and row `other` with wo.
-  auto source = [&](bool valid, int i, int other, float wr, float wo) {
+  // Query i's member reads row r with weight wr and row `other` with wo;
+  // offset members carry query i's log-prior.
+  auto source = [&](bool valid, int i, int other, float wr, float wo, bool off) {
     const int ii = valid ? i : 0;
     float q1[N], q2[N], g1[N], g2[N];
     load_krot<T, D>(Q, a.rope, ii, j0, q1, q2);
@@ -379,7 +390,7 @@ __global__ void __launch_bounds__(kGenWarps * 32) k_bwd_kv_general(const GenArgs
       s_part += q1[h] * key1[h] + q2[h] * key2[h];
       dp_part += g1[h] * val1[h] + g2[h] * val2[h];
     }
-    const float s = group8_sum(s_part);
+    const float s = group8_sum(s_part) + ((off && a.beta) ? __ldg(a.beta + (size_t)unit * a.T + ii) : 0.f);
     const float dp = group8_sum(dp_part);
     if (valid) {
       const float p = expf(s - __ldg(lse + ii));
@@ -393,15 +404,15 @@ __global__ void __launch_bounds__(kGenWarps * 32) k_bwd_kv_general(const GenArgs
     }
   };
 
-  for (int t = 0; t < a.W; ++t) source(active && rr + t < a.T, rr + t, -1, 1.f, 0.f);
+  for (int t = 0; t < a.W; ++t) source(active && rr + t < a.T, rr + t, -1, 1.f, 0.f, false);
   for (int k = 0; k < a.n_off; ++k) {
     const OffGeo g = sg[k];
     if (!g.ok) continue;                                     // CTA-uniform
     const int ia = rr + g.lo;                                // r is row a
-    source(active && ia < a.T && ia - g.c >= 0, ia, g.w != 0.f ? rr - 1 : -1, g.wa, g.w);
+    source(active && ia < a.T && ia - g.c >= 0, ia, g.w != 0.f ? rr - 1 : -1, g.wa, g.w, true);
     if (g.w != 0.f) {                                        // r is row b
       const int ib = rr + g.lo + 1;
-      source(active && ib < a.T, ib, rr + 1, g.w, g.wa);
+      source(active && ib < a.T, ib, rr + 1, g.w, g.wa, true);
     }
   }
   if (active && rr < a.S) {
@@ -503,7 +514,7 @@ template <typename T, int D>
 static cudaError_t fwd_t(const Problem& pb, const FwdPtrs& p, cudaStream_t st) {
   GenArgs a = make_args(pb);
   a.q = p.q; a.k = p.k; a.v = p.v; a.alpha = p.alpha; a.rope = p.rope;
-  a.out_o = p.o; a.out_lse = p.lse;
+  a.out_o = p.o; a.out_lse = p.lse; a.beta = p.beta;
   const long long grid = (long long)pb.units() * a.n_tiles;
   trace_mark("fwd_general", st, true);
   k_fwd_general<T, D><<<(unsigned)grid, kGenWarps * 32, 0, st>>>(a);
@@ -519,6 +530,7 @@ static cudaError_t bwd_t(const Problem& pb, const BwdPtrs& p, cudaStream_t st, i
   a.q = p.q; a.k = p.k; a.v = p.v; a.o = p.o; a.dout = p.dout; a.lse = p.lse;
   a.alpha = p.alpha; a.rope = p.rope;
   a.dq = p.dq; a.dk = p.dk; a.dv = p.dv;
+  a.beta = p.beta; a.dbeta = p.dbeta;
   a.dvec = reinterpret_cast<float*>(ws + lay.d_off);
   a.dal_part = reinterpret_cast<float*>(ws + lay.dal_off);
   a.sink_k = reinterpret_cast<float*>(ws + lay.sink_off);

@@ -23,6 +23,7 @@ struct FwdPtrs {
   const float* alpha;
   void* o; float* lse;
   const float2* rope;           // [T_cap][D/2] (cos, sin)
+  const float* beta;            // log-prior on offset members [units][T], or nullptr
 };
 
 struct BwdPtrs {
@@ -31,6 +32,8 @@ struct BwdPtrs {
   void* dq; void* dk; void* dv; float* dalpha;
   const float2* rope;
   void* workspace;
+  const float* beta;            // log-prior on offset members [units][T], or nullptr
+  float* dbeta;                 // its gradient [units][T], or nullptr
 };
 
 // Workspace carving of the general backward (offsets in bytes).

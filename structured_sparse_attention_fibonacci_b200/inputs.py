@@ -53,6 +53,7 @@ class Workload:
     seed: int                  # layer l uses seed + l (the tiny case: seed 0 for all)
     backward: bool = False
     decode: bool = False       # one new token at position T - 1 against a T-row KV cache
+    prior: bool = False        # a per-query log-prior beta on the offset members
     offsets: Tuple[int, ...] = FIB15
     rope_base: float = 10000.0
     note: str = ""
@@ -96,6 +97,13 @@ WORKLOADS = {
                              "current and 4 previous keys plus one skip to i - 16 (k = 4, "
                              "pi = 16, the best setting of the pi-Attention page), 16 layers "
                              "B=8 H=8 T=1024 d=64 bf16"),
+    "pi_gate_train": Workload("pi_gate_train", 16, 8, 8, 1024, 64, 5, 0, torch.bfloat16, "fixed",
+                              8000, backward=True, prior=True, offsets=(16,),
+                              note="the periodic-skip pattern with pi-Attention's fusion of "
+                                   "local and skip logits in one softmax: a per-query "
+                                   "log-prior beta ~ N(0, 1) on the skip member, forward and "
+                                   "backward (dQ, dK, dV, dbeta), 16 layers B=8 H=8 T=1024 "
+                                   "d=64 bf16, W=5, offset 16"),
     "decode_4k": Workload("decode_4k", 16, 8, 8, 4096, 64, 12, 0, torch.bfloat16, "linear", 6000,
                           decode=True,
                           note="single-token decode: 16 layers B=8 H=8 d=64 bf16, one new query "
@@ -152,3 +160,17 @@ def make_decode_inputs(wl: Workload, device: Optional[str] = None, pin: bool = F
     if device is not None:
         q, k, v = q.to(device), k.to(device), v.to(device)
     return q, k, v
+
+
+def make_prior(wl: Workload, device: Optional[str] = None, layers: Optional[range] = None,
+               pin: bool = False):
+    """The log-prior beta [L, B, H, T] of a workload with ``prior``: layer l
+    draws N(0, 1) values in fp32 from a CPU generator seeded with
+    ``seed + 500000 + l`` (the gate logits a fusion network would produce,
+    here synthetic)."""
+    layers = range(wl.L) if layers is None else layers
+    out = torch.empty((len(layers), wl.B, wl.H, wl.T), dtype=torch.float32, pin_memory=pin)
+    for li, l in enumerate(layers):
+        g = torch.Generator(device="cpu").manual_seed(wl.seed + 500000 + l)
+        out[li].copy_(torch.randn((wl.B, wl.H, wl.T), generator=g, dtype=torch.float32))
+    return out if device is None else out.to(device)
