@@ -157,11 +157,12 @@ __device__ __forceinline__ void window_axpy(const unsigned char* ring, int RB, i
   }
 }
 
+// Window lags in blocks of 4: the unrolled body stays small enough for the
+// instruction cache (measured on B200: 8-lag blocks ran 5-14% slower).
 #define SA_WINDOW_CHUNKS(W, CALL)                                   \
   {                                                                 \
     int d0 = 0;                                                     \
-    while ((W) - d0 >= 8) { CALL(8); d0 += 8; }                     \
-    if ((W) - d0 >= 4) { CALL(4); d0 += 4; }                        \
+    while ((W) - d0 >= 4) { CALL(4); d0 += 4; }                     \
     if ((W) - d0 >= 2) { CALL(2); d0 += 2; }                        \
     if ((W) - d0 >= 1) { CALL(1); d0 += 1; }                        \
   }
@@ -646,7 +647,7 @@ __device__ __forceinline__ int key_pass(const FastBwdArgs& a, Stager& stg, unsig
   // window: key rg+kk takes query row rg+d0+u at lag d0 + u - kk
   int d0 = 0;
   while (d0 < W) {
-    const int LCr = W - d0 >= 8 ? 8 : (W - d0 >= 4 ? 4 : (W - d0 >= 2 ? 2 : 1));
+    const int LCr = W - d0 >= 4 ? 4 : (W - d0 >= 2 ? 2 : 1);
 #define SA_KEY_WINDOW(LC)                                                           \
     {                                                                               \
       float wl[LC][4];                                                              \
@@ -665,8 +666,7 @@ __device__ __forceinline__ int key_pass(const FastBwdArgs& a, Stager& stg, unsig
         }                                                                           \
       }                                                                             \
     }
-    if (LCr == 8) SA_KEY_WINDOW(8)
-    else if (LCr == 4) SA_KEY_WINDOW(4)
+    if (LCr == 4) SA_KEY_WINDOW(4)
     else if (LCr == 2) SA_KEY_WINDOW(2)
     else SA_KEY_WINDOW(1)
 #undef SA_KEY_WINDOW
