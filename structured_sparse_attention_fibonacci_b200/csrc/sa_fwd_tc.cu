@@ -493,7 +493,24 @@ bool tc_fwd_supported(const Problem& pb) {
          tc_fwd_smem(pb, nullptr, nullptr) <= 200 * 1024;
 }
 
-bool tc_fwd_preferred(const Problem& pb) { return tc_fwd_supported(pb) && pb.W >= 32; }
+// CTAs of `smem` dynamic bytes that share one SM's 228 KB (1 KB reserved per
+// CTA plus about 1 KB of static shared memory), at most the 4 of the
+// launch bounds.
+static int ctas_per_sm(size_t smem) {
+  const size_t per = smem + 2048;
+  return (int)std::min<size_t>(4, (size_t)(228 * 1024) / per);
+}
+
+// Measured on B200 (B=1 H=16 T=32768 with 4 sinks, and B=2 H=8 T=4096):
+// - the tensor-core forward is faster from W = 32 up (by 18-38% at W = 64..112);
+// - it is slower where its larger ring leaves it one CTA per SM and the
+//   CUDA-core forward keeps two (W = 128: 0.95 vs 0.87 ms).
+bool tc_fwd_preferred(const Problem& pb) {
+  if (!tc_fwd_supported(pb) || pb.W < 32) return false;
+  const int tc = ctas_per_sm(tc_fwd_smem(pb, nullptr, nullptr));
+  const int cc = fast_fwd_supported(pb) ? ctas_per_sm(fast_fwd_smem(pb, nullptr, nullptr)) : 0;
+  return !(tc == 1 && cc >= 2);
+}
 
 cudaError_t launch_fwd_tc(const Problem& pb, const FwdPtrs& p, void* keys_ws, cudaStream_t st,
                           int* launches) {

@@ -73,9 +73,9 @@ cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& a, void* keys_ws, 
 // Tensor-core bf16 / D=64 forward (sa_fwd_tc.cu); keys_ws as for the staged
 // forward (fast_fwd_workspace bytes, required).
 bool tc_fwd_supported(const Problem& pb);
-// Where the tensor-core forward is the faster one (long windows: measured on
-// B200, W = 64 runs 11% faster than the CUDA-core forward, W = 12 breaks even
-// on T = 1024 and is 8% slower on T = 4096).
+// Where the tensor-core forward is the faster one: windows of 32 and more,
+// except where its shared memory leaves it one CTA per SM while the CUDA-core
+// forward keeps two (measured on B200; W = 12 is 9% slower on tensor cores).
 bool tc_fwd_preferred(const Problem& pb);
 size_t tc_fwd_smem(const Problem& pb, int* ring_rows, int* sc_stride);
 cudaError_t launch_fwd_tc(const Problem& pb, const FwdPtrs& a, void* keys_ws, cudaStream_t st,
