@@ -88,6 +88,8 @@ def test_workspace_sizes(lib):
     (dict(sinks=-1), sa.SA_ERR_INVALID_ARG),
     (dict(sinks=17), sa.SA_ERR_UNSUPPORTED),
     (dict(rope_base=0.0), sa.SA_ERR_INVALID_ARG),
+    (dict(shape=(1, 1, 1, (1 << 24) + 1, 64)), sa.SA_ERR_UNSUPPORTED),   # beyond the position range
+    (dict(shape=(4096, 64, 64, 1 << 20, 64)), sa.SA_ERR_UNSUPPORTED),     # grid beyond 2^31 CTAs
 ])
 def test_bad_params_rejected_on_host(lib, bad, code):
     p = _p(**bad)

@@ -269,3 +269,40 @@ def test_fast_backward_is_the_one_dispatched():
         sa.trace_enable(False)
     assert names == {"rope_keys", "rope_queries", "bwd_q_fast", "bwd_kv_fast",
                      "reduce_dalpha"}, names
+
+
+def test_tensors_beyond_2_31_elements():
+    """Maximum sizes: 520 (layer, batch, head) units of T = 65536 rows of 64
+    (2.2e9 elements per tensor, 4.4 GB in bf16). The last unit starts past
+    element 2^31, so any 32-bit index arithmetic would show. Units 0 and 519
+    hold N(0, 1) data; every other unit is zero. Zero units contribute nothing
+    to any output or to dalpha: q = k = v = dO = 0 there. So the oracle on the
+    two data units gives the whole expected result. That covers O and LSE,
+    dQ, dK and dV of those units, and the layer's dalpha, through the staged
+    forward and backward."""
+    L, B, H, T, D = 1, 1, 520, 65536, 64
+    shape = (L, B, H, T, D)
+    assert L * B * H * T * D > 2 ** 31
+    data_units = (0, H - 1)
+    g = torch.Generator(device="cpu").manual_seed(2031)
+    host = {u: [torch.randn((T, D), generator=g, dtype=torch.float32).to(torch.bfloat16)
+                for _ in range(4)] for u in data_units}
+    q, k, v, do = (torch.zeros(shape, dtype=torch.bfloat16, device=DEV) for _ in range(4))
+    for u in data_units:
+        for t, x in zip((q, k, v, do), host[u]):
+            t[0, 0, u].copy_(x)
+    alpha = torch.tensor([1.1234], device=DEV)
+    kw = dict(window=12, sinks=0, offsets=FIB15)
+    o, lse = sa.fwd(q, k, v, alpha, **kw)
+    dq, dk, dv, dal = sa.bwd(q, k, v, o, lse, do, alpha, **kw)
+    torch.cuda.synchronize()
+    assert sa.device_error() == 0
+    sel = lambda t: t[:, :, list(data_units)].contiguous()
+    o_ref, lse_ref = oracle_fwd(sel(q), sel(k), sel(v), alpha, **kw)
+    check_fwd(sel(o), sel(lse), o_ref, lse_ref, torch.bfloat16, "beyond 2^31 forward")
+    ref = oracle_bwd(sel(q), sel(k), sel(v), sel(do), alpha, **kw)
+    check_bwd((sel(dq), sel(dk), sel(dv), dal), ref, torch.bfloat16, "beyond 2^31 backward")
+    # a zero unit in between: zero outputs and gradients
+    mid = H // 2
+    for t in (o, dq, dk, dv):
+        assert t[0, 0, mid].float().abs().max().item() == 0.0
