@@ -785,6 +785,8 @@ __global__ void __launch_bounds__(kFastM, 4) k_bwd_kv_fast(const FastBwdArgs a) 
       if (r < T && r < S) {
         const size_t per = (size_t)S * kD;
         const float* src = sink + (size_t)unit * a.n_tiles * per + (size_t)r * kD;
+        // two tiles' loads in flight (the sum stays in tile order)
+#pragma unroll 2
         for (int tt = 0; tt < a.n_tiles; ++tt) {
 #pragma unroll
           for (int h = 0; h < 8; ++h) {

@@ -419,6 +419,8 @@ __global__ void __launch_bounds__(kGenWarps * 32) k_bwd_kv_general(const GenArgs
     const size_t per = (size_t)a.S * D;
     const float* gk = a.sink_k + (size_t)unit * a.n_tiles * per + (size_t)rr * D;
     const float* gv = a.sink_v + (size_t)unit * a.n_tiles * per + (size_t)rr * D;
+    // four tiles' loads in flight (the sum stays in tile order)
+#pragma unroll 4
     for (int t = 0; t < a.n_tiles; ++t) {
 #pragma unroll
       for (int h = 0; h < N; ++h) {
