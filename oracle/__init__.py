@@ -61,7 +61,7 @@ class Oracle:
                             ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
             dec = getattr(lib, "oracle_decode" + suffix)
             dec.restype = ctypes.c_int
-            dec.argtypes = head + [ctypes.c_int64] + [P] * 5
+            dec.argtypes = head + [ctypes.c_int64] + [P] * 6
             a_th = getattr(lib, "oracle_alpha_from_theta" + suffix)
             a_th.restype = None
             a_th.argtypes = [ctypes.c_int, P, P]
@@ -132,9 +132,11 @@ class Oracle:
         return (dq, dk, dv, dal, dbt) if beta is not None else (dq, dk, dv, dal)
 
     def decode(self, q1, k, v, alpha, pos, *, window, offsets=FIB15, sinks=0,
-               rope_base=10000.0, scale=0.0, precision="f64"):
+               rope_base=10000.0, scale=0.0, precision="f64", beta=None):
         """Single-token decode: q1 [L, B, H, D] at position pos against the
-        caches k, v [L, B, H, T, D] (rows 0..pos used).  Returns (O1, LSE1)."""
+        caches k, v [L, B, H, T, D] (rows 0..pos used).  beta: optional
+        [L, B, H] log-prior on the new query's offset members.
+        Returns (O1, LSE1)."""
         dt, ct = _np_dtype(precision)
         q1, k, v = (_prep(x, dt) for x in (q1, k, v))
         L, B, H, T, D = k.shape
@@ -144,10 +146,12 @@ class Oracle:
         offs = np.ascontiguousarray(np.asarray(offsets, dtype=np.int32).reshape(-1))
         o = np.empty_like(q1)
         lse = np.empty((L, B, H), dtype=dt)
+        bt = _prep(beta, dt).reshape(L, B, H) if beta is not None else None
         fn = getattr(self.lib, "oracle_decode_" + precision)
         rc = fn(L, B, H, T, D, int(window), len(offs), _ptr(offs, ctypes.c_int32), int(sinks),
                 float(rope_base), float(scale), _ptr(al, ctypes.c_float), int(pos),
-                _ptr(q1, ct), _ptr(k, ct), _ptr(v, ct), _ptr(o, ct), _ptr(lse, ct))
+                _ptr(q1, ct), _ptr(k, ct), _ptr(v, ct), _ptr(o, ct), _ptr(lse, ct),
+                _ptr(bt, ct) if bt is not None else None)
         if rc != 0:
             raise ValueError(f"oracle_decode rejected its arguments (rc={rc})")
         return o, lse

@@ -397,12 +397,13 @@ int FN(oracle_bwd)(int L, int B, int H, int T, int D, int W, int n_off,
  * "Attended set"; rows after pos are never touched).  Q1 and O1 are
  * [L][B][H][D]; K and V are [L][B][H][T][D] with pos < T; LSE1 is
  * [L][B][H] (may be NULL).  Each key row a member reads is rotated at its own
- * position, one member at a time.
+ * position, one member at a time.  beta1 (may be NULL): the new query's
+ * log-prior on its offset members, [L][B][H].
  */
 int FN(oracle_decode)(int L, int B, int H, int T, int D, int W, int n_off,
                       const int32_t* offsets, int S, double rope_base, double scale,
                       const float* alpha, int64_t pos, const real* Q1, const real* K,
-                      const real* V, real* O1, real* LSE1) {
+                      const real* V, real* O1, real* LSE1, const real* beta1) {
   prob_t p = {L, B, H, T, D, W, n_off, S, rope_base, scale, offsets, alpha};
   if (check(&p) || pos < 0 || pos >= T) return -1;
   const double s = scale > 0 ? scale : 1.0 / sqrt((double)D);
@@ -435,6 +436,7 @@ int FN(oracle_decode)(int L, int B, int H, int T, int D, int W, int n_off,
         rope_row(Ku + mb[m].b * D, mb[m].b, D, rope_base, kb);
         v += mb[m].wb * dot(qh, kb, D);
       }
+      if (beta1 && mb[m].kind == 2) v += beta1[u];   /* log-prior */
       sc[m] = v;
       if (v > mx) mx = v;
     }

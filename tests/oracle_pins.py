@@ -335,6 +335,13 @@ def pin_decode_dense_and_gather(orc):
                              [alpha], window=5, sinks=1, offsets=FIB)
             _close(o, of[..., pos, :], 1e-12, what=f"decode vs forward alpha={alpha}")
             _close(lse, lf[..., pos], 1e-12, what=f"decode vs forward LSE alpha={alpha}")
+        # with a log-prior: row pos of the forward whose query pos has that prior
+        beta = _rand((L, B, H, pos + 1), 73 + pos)
+        o, lse = orc.decode(q1, kc, vc, [0.91], pos, window=4, offsets=FIB, beta=beta[..., pos])
+        of, lf = orc.fwd(q[..., :pos + 1, :], k[..., :pos + 1, :], v[..., :pos + 1, :], [0.91],
+                         window=4, offsets=FIB, beta=beta)
+        _close(o, of[..., pos, :], 1e-12, what=f"decode with a prior pos={pos}")
+        _close(lse, lf[..., pos], 1e-12, what=f"decode with a prior, LSE pos={pos}")
 
 
 # -- log-prior on the offset members (pi-Attention's fusion in one softmax) ---

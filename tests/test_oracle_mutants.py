@@ -50,6 +50,8 @@ MUTANTS = [
      "sc[m] = dot(qh, krow + m * D, D);\n        if (beta && mb[m].kind == 99)"),
     ("dbeta_all_members", "if (mb[m].kind == 2) dbet += gs;", "dbet += gs;"),
     ("dbeta_uses_p", "if (mb[m].kind == 2) dbet += gs;", "if (mb[m].kind == 2) dbet += pm;"),
+    ("decode_prior_on_window", "if (beta1 && mb[m].kind == 2) v += beta1[u];",
+     "if (beta1 && mb[m].kind != 1) v += beta1[u];"),
     ("decode_query_scale", "for (int d = 0; d < D; ++d) qh[d] = (real)s * qh[d];\n    int n = members_of(pos",
      "for (int d = 0; d < D; ++d) qh[d] = qh[d];\n    int n = members_of(pos"),
 ]
