@@ -179,16 +179,16 @@ sa_status sparse_attn_bwd_ctx(const sa_params* p, const void* q, const void* k, 
  *           dLoss/dbeta_i = sum over query i's offset members of dLoss/dscore
  *                                                                 (written)
  * sparse_attn_fwd_prior: arguments as sparse_attn_fwd plus beta. context
- *   NULL runs the plain forward. The bf16 / D = 64 configurations then use
- *   the CUDA-core staged kernel whatever sparse_attn_select_forward says:
- *   the tensor-core forward has no prior. A non-NULL context runs the training
- *   forward (as sparse_attn_fwd_train): the saved probabilities include the
- *   prior, and workspace is unused.
+ *   NULL runs the plain forward, with the same kernel choice as
+ *   sparse_attn_fwd. A non-NULL context runs the training forward (as
+ *   sparse_attn_fwd_train): the saved probabilities include the prior, and
+ *   workspace is unused.
  * sparse_attn_bwd_prior: arguments as sparse_attn_bwd plus beta (the
  *   forward's), an optional context (from sparse_attn_fwd_prior with the same
  *   beta; lse may then be NULL) and dbeta.
- * beta, dbeta: non-NULL, 4-byte aligned, else SA_ERR_INVALID_ARG.  Decode and
- * the allocation-free forward take no prior.
+ * beta, dbeta: non-NULL, 4-byte aligned, else SA_ERR_INVALID_ARG.  Decode
+ * takes the prior through sparse_attn_decode_prior; the allocation-free
+ * forward takes none.
  */
 sa_status sparse_attn_fwd_prior(const sa_params* p, const void* q, const void* k, const void* v,
                                 const float* alpha, const float* beta, void* o, float* lse,
@@ -221,6 +221,14 @@ sa_status sparse_attn_bwd_prior(const sa_params* p, const void* q, const void* k
 sa_status sparse_attn_decode(const sa_params* p, int32_t pos, const void* q, const void* k,
                              const void* v, const float* alpha, void* o, float* lse,
                              void* stream);
+/*
+ * Decode with the log-prior of sparse_attn_fwd_prior: beta is the new
+ * queries' prior, device fp32 [L][B][H], added to the score of each of their
+ * offset members. NULL means none, as in sparse_attn_decode.
+ */
+sa_status sparse_attn_decode_prior(const sa_params* p, int32_t pos, const void* q, const void* k,
+                                   const void* v, const float* alpha, const float* beta, void* o,
+                                   float* lse, void* stream);
 
 /*
  * Learned-alpha parametrisation.  The page trains "one free parameter theta

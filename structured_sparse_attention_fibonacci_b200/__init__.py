@@ -35,7 +35,7 @@ EXPORTED = ("sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_workspace_size",
             "sparse_attn_fwd_noalloc", "sparse_attn_device_error", "sparse_attn_select_forward",
             "sparse_attn_context_size", "sparse_attn_fwd_train", "sparse_attn_bwd_ctx",
             "sparse_attn_decode", "sparse_attn_alpha_from_theta", "sparse_attn_dtheta",
-            "sparse_attn_fwd_prior", "sparse_attn_bwd_prior")
+            "sparse_attn_fwd_prior", "sparse_attn_bwd_prior", "sparse_attn_decode_prior")
 
 
 class SaParams(ctypes.Structure):
@@ -87,6 +87,8 @@ def lib():
         L.sparse_attn_dtheta.argtypes = [ctypes.c_int32, fp, fp, fp, vp]
         L.sparse_attn_decode.restype = ctypes.c_int
         L.sparse_attn_decode.argtypes = [P, ctypes.c_int32, vp, vp, vp, fp, vp, fp, vp]
+        L.sparse_attn_decode_prior.restype = ctypes.c_int
+        L.sparse_attn_decode_prior.argtypes = [P, ctypes.c_int32, vp, vp, vp, fp, fp, vp, fp, vp]
         L.sparse_attn_context_size.restype = ctypes.c_size_t
         L.sparse_attn_context_size.argtypes = [P]
         L.sparse_attn_fwd_train.restype = ctypes.c_int
@@ -314,10 +316,13 @@ def dtheta(theta, dalpha, out=None, stream=None):
 
 
 def decode(q, k_cache, v_cache, alpha, pos, *, window, offsets=FIB15, sinks=0,
-           rope_base=10000.0, scale=0.0, out=None, lse=None, want_lse=True, stream=None):
+           rope_base=10000.0, scale=0.0, out=None, lse=None, want_lse=True, stream=None,
+           beta=None):
     """Single-token decode: q [L, B, H, D] at position pos against the caches
     k_cache, v_cache [L, B, H, T_cache, D] (rows 0..pos hold the sequence,
-    row pos the new token).  Returns (O [L, B, H, D], LSE [L, B, H] or None)."""
+    row pos the new token).  beta: optional CUDA fp32 [L, B, H] log-prior on
+    the new queries' offset members.  Returns (O [L, B, H, D], LSE [L, B, H]
+    or None)."""
     shape = tuple(k_cache.shape)
     dtype, dev = k_cache.dtype, k_cache.device
     if tuple(q.shape) != shape[:3] + shape[4:]:
@@ -330,10 +335,13 @@ def decode(q, k_cache, v_cache, alpha, pos, *, window, offsets=FIB15, sinks=0,
         lse = torch.empty(shape[:3], dtype=torch.float32, device=dev)
     p = make_params(shape, dtype, window=window, offsets=offsets, sinks=sinks,
                     rope_base=rope_base, scale=scale)
-    st = lib().sparse_attn_decode(ctypes.byref(p), int(pos), _ptr(q), _ptr(k_cache),
-                                  _ptr(v_cache), _ptr(alpha), _ptr(out), _ptr(lse),
-                                  _stream_handle(stream))
-    _check("sparse_attn_decode", st)
+    if beta is not None and (beta.device != dev or not beta.is_contiguous()
+                             or beta.dtype != torch.float32 or tuple(beta.shape) != shape[:3]):
+        raise ValueError(f"beta must be a contiguous CUDA fp32 tensor of shape {shape[:3]}")
+    st = lib().sparse_attn_decode_prior(ctypes.byref(p), int(pos), _ptr(q), _ptr(k_cache),
+                                        _ptr(v_cache), _ptr(alpha), _ptr(beta), _ptr(out),
+                                        _ptr(lse), _stream_handle(stream))
+    _check("sparse_attn_decode_prior", st)
     return out, lse
 
 

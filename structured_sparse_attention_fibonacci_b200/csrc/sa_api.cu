@@ -228,9 +228,9 @@ sa_status fwd_impl(const sa_params* p, const void* q, const void* k, const void*
   cudaError_t e;
   if (g_force_general || !sa::fast_fwd_supported(pb))
     e = sa::launch_fwd_general(pb, a, st, &launches);
-  else if (!beta && (g_fwd_select == 2 ? sa::tc_fwd_supported(pb)
-                                       : (g_fwd_select == 0 && sa::tc_fwd_preferred(pb))))
-    e = sa::launch_fwd_tc(pb, a, workspace, st, &launches);   // (no log-prior there)
+  else if (g_fwd_select == 2 ? sa::tc_fwd_supported(pb)
+                              : (g_fwd_select == 0 && sa::tc_fwd_preferred(pb)))
+    e = sa::launch_fwd_tc(pb, a, workspace, st, &launches);
   else
     e = sa::launch_fwd_fast(pb, a, workspace, st, &launches);
   if (e != cudaSuccess) return SA_ERR_CUDA;
@@ -347,18 +347,24 @@ sa_status sparse_attn_bwd_prior(const sa_params* p, const void* q, const void* k
 sa_status sparse_attn_decode(const sa_params* p, int32_t pos, const void* q, const void* k,
                              const void* v, const float* alpha, void* o, float* lse,
                              void* stream) {
+  return sparse_attn_decode_prior(p, pos, q, k, v, alpha, nullptr, o, lse, stream);
+}
+
+sa_status sparse_attn_decode_prior(const sa_params* p, int32_t pos, const void* q, const void* k,
+                                   const void* v, const float* alpha, const float* beta, void* o,
+                                   float* lse, void* stream) {
   sa::Problem pb;
   sa_status s = build_problem(p, &pb);
   if (s != SA_OK) return s;
   if (pos < 0 || pos >= pb.T) return SA_ERR_INVALID_ARG;
   if (!q || !k || !v || !alpha || !o) return SA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (lse && !aligned4(lse)) || !aligned4(alpha))
+      (lse && !aligned4(lse)) || !aligned4(alpha) || (beta && !aligned4(beta)))
     return SA_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const float2* rope = nullptr;
   if ((s = rope_table(pb.T, pb.D, p->rope_base, st, &rope)) != SA_OK) return s;
-  if (sa::launch_decode(pb, pos, q, k, v, alpha, rope, o, lse, st) != cudaSuccess)
+  if (sa::launch_decode(pb, pos, q, k, v, alpha, rope, o, lse, st, beta) != cudaSuccess)
     return SA_ERR_CUDA;
   g_last_launches = 1;
   return SA_OK;

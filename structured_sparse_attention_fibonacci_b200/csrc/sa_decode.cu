@@ -30,6 +30,7 @@ struct DecArgs {
   const void* q; const void* k; const void* v;
   const float* alpha; const float2* rope;
   void* o; float* lse;
+  const float* beta;                   // log-prior on the offset members [units], or nullptr
 };
 
 // q_hat . RoPE(K[row]) over D dims; q_hat in shared memory.
@@ -144,7 +145,9 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(const DecArgs a) {
     }
     sw[m] = s;
   }
-  // offsets: lane k's geometry, so the offset members go by lane
+  // offsets: lane k's geometry, so the offset members go by lane; each
+  // carries the query's log-prior (0 without one)
+  const float prior = a.beta ? __ldg(a.beta + unit) : 0.f;
   for (int k0 = 0; k0 < n_off; k0 += 32) {
     const int k = k0 + lane;
     if (k < n_off) {
@@ -152,6 +155,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(const DecArgs a) {
       if (pos - og.c >= 0) {
         s = og.wa * key_dot<T, D>(K, a.rope, pos - og.lo, sq);
         if (og.w != 0.f) s += og.w * key_dot<T, D>(K, a.rope, pos - og.lo - 1, sq);
+        s += prior;
       }
       sw[W + S + k] = s;
     }
@@ -239,12 +243,13 @@ cudaError_t launch_t(const DecArgs& a, long long units, cudaStream_t st) {
 
 cudaError_t launch_decode(const Problem& pb, int pos, const void* q, const void* k, const void* v,
                           const float* alpha, const float2* rope, void* o, float* lse,
-                          cudaStream_t st) {
+                          cudaStream_t st, const float* beta) {
   DecArgs a = {};
   a.B = pb.B; a.H = pb.H; a.Tc = pb.T; a.W = pb.W; a.n_off = pb.n_off; a.S = pb.S; a.pos = pos;
   a.scale = pb.scale;
   for (int j = 0; j < pb.n_off; ++j) a.f[j] = pb.f[j];
   a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.rope = rope; a.o = o; a.lse = lse;
+  a.beta = beta;
   const long long units = pb.units();
   a.units = units;
   const bool f32 = pb.dtype == SA_DTYPE_F32;

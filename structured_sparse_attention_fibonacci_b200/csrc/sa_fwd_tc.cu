@@ -47,6 +47,7 @@ struct TcFwdArgs {
   const float* alpha; const float2* rope;
   __nv_bfloat16* o; float* lse;
   unsigned* err;
+  const float* beta;                   // log-prior on offset members [units][T], or nullptr
 };
 
 enum : int { kFar = 0, kNear = 1, kDead = 2 };
@@ -296,12 +297,18 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
     const int i = i0 + t;
     float* my = sc + (size_t)t * st;
     if (i < T) {
-      for (int k = 0; k < n_off; ++k) {       // near offsets: from two window scores
-        if (s_kind[k] != kNear) continue;
-        const OffGeo og = sg[k];
-        float sv = og.wa * my[og.lo];
-        if (og.w != 0.f) sv += og.w * my[og.lo + 1];
-        my[W + S + k] = sv;
+      // near offsets from two window scores; every offset member gets the
+      // query's log-prior (0 without one)
+      const float prior = a.beta ? __ldg(a.beta + (size_t)unit * T + i) : 0.f;
+      for (int k = 0; k < n_off; ++k) {
+        if (s_kind[k] == kNear) {
+          const OffGeo og = sg[k];
+          float sv = og.wa * my[og.lo];
+          if (og.w != 0.f) sv += og.w * my[og.lo + 1];
+          my[W + S + k] = sv + prior;
+        } else if (s_kind[k] == kFar) {
+          my[W + S + k] += prior;
+        }
       }
       float mx = -INFINITY;
       for (int d = 0; d < W; ++d)
@@ -523,7 +530,7 @@ cudaError_t launch_fwd_tc(const Problem& pb, const FwdPtrs& p, void* keys_ws, cu
   std::sort(a.f, a.f + pb.n_off);
   const size_t smem = tc_fwd_smem(pb, &a.ring_rows, &a.sc_stride);
   a.q = reinterpret_cast<const __nv_bfloat16*>(p.q);
-  a.alpha = p.alpha; a.rope = p.rope;
+  a.alpha = p.alpha; a.beta = p.beta; a.rope = p.rope;
   a.o = reinterpret_cast<__nv_bfloat16*>(p.o); a.lse = p.lse;
   cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&a.err), g_fwd_tc_err);
   if (e != cudaSuccess) return e;

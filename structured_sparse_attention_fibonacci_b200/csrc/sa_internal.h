@@ -127,9 +127,10 @@ cudaError_t launch_alpha_from_theta(int L, const float* theta, float* alpha, cud
 cudaError_t launch_dtheta(int L, const float* theta, const float* dalpha, float* dtheta,
                           cudaStream_t st);
 // Single-token decode (sa_decode.cu): pb.T is the cache length, pos < pb.T.
+// beta: the new queries' log-prior on their offset members [units], or nullptr.
 cudaError_t launch_decode(const Problem& pb, int pos, const void* q, const void* k, const void* v,
                           const float* alpha, const float2* rope, void* o, float* lse,
-                          cudaStream_t st);
+                          cudaStream_t st, const float* beta = nullptr);
 cudaError_t launch_fwd_general(const Problem& pb, const FwdPtrs& a, cudaStream_t st, int* launches);
 cudaError_t launch_bwd_general(const Problem& pb, const BwdPtrs& a, cudaStream_t st, int* launches);
 

@@ -120,3 +120,24 @@ def test_decode_workload_full_size():
         o_ref, lse_ref = oracle.decode(to_np(q1[l:l + 1]), to_np(kc[l:l + 1]), to_np(vc[l:l + 1]),
                                        alpha[l:l + 1].numpy(), wl.T - 1, **kw)
         check_fwd(o[l:l + 1], lse[l:l + 1], o_ref, lse_ref, wl.dtype, f"decode_4k layer {l}")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("case", [c for c in CASES if c[0] in ("bf16_d64_stagger", "fp32_d32_learned")],
+                         ids=lambda c: c[0])
+def test_decode_with_a_prior(case):
+    """sparse_attn_decode_prior: the new queries' log-prior on their offset
+    members, against the oracle's decode with the same prior."""
+    name, dtype, shape, W, S, alphas, offs, positions = case
+    q, k, v = _caches(shape, dtype, zlib.crc32(name.encode()) % 10000 + 1)
+    g = torch.Generator(device="cpu").manual_seed(44)
+    beta = 1.5 * torch.randn(shape[:3], generator=g)
+    alpha = torch.tensor(alphas, dtype=torch.float32)
+    kw = dict(window=W, sinks=S, offsets=offs)
+    for pos in positions:
+        o, lse = sa.decode(q.to(DEV), k.to(DEV), v.to(DEV), alpha.to(DEV), pos, beta=beta.to(DEV),
+                           **kw)
+        torch.cuda.synchronize()
+        o_ref, lse_ref = oracle.decode(to_np(q), to_np(k), to_np(v), alpha.numpy(), pos,
+                                       beta=beta.numpy(), **kw)
+        check_fwd(o, lse, o_ref, lse_ref, dtype, f"{name} prior pos={pos}")

@@ -9,8 +9,8 @@ sparse_attn_bwd_prior through the C ABI.
 
 Paths covered:
 - the general kernels: fp32, and bf16 with D != 64;
-- the staged CUDA-core kernels: bf16, D = 64, including a window of 64,
-  where the plain forward would take the tensor-core kernel;
+- the staged kernels: bf16, D = 64, both forwards (CUDA-core and
+  tensor-core) and the backward;
 - the training pair with a context;
 - the general kernels forced on a staged configuration.
 
@@ -134,18 +134,27 @@ def test_prior_general_kernels_forced():
 
 
 @pytest.mark.gpu
-def test_prior_skips_the_tensor_core_forward():
-    """W = 64 would take the tensor-core forward; with a prior the CUDA-core
-    staged forward runs (it carries the prior)."""
+@pytest.mark.parametrize("kernel", [1, 2])
+def test_prior_on_both_staged_forwards(kernel):
+    """W = 64 with sinks: the tensor-core forward (the default there) and the
+    CUDA-core forward both carry the prior; each is dispatched as selected and
+    matches the oracle."""
     q, k, v, do, beta = _inputs((1, 1, 2, 300, 64), torch.bfloat16, 5, 1.0)
-    alpha = torch.ones(1, device=DEV)
-    sa.trace_enable(True)
-    sa.trace_read()
-    sa.fwd(q, k, v, alpha, beta=beta, window=64, sinks=4)
-    torch.cuda.synchronize()
-    names = set(sa.trace_read())
-    sa.trace_enable(False)
-    assert "fwd_fast" in names and "fwd_tc" not in names, names
+    alpha = torch.tensor([1.1], device=DEV)
+    kw = dict(window=64, sinks=4)
+    sa.select_forward(kernel)
+    try:
+        sa.trace_enable(True)
+        sa.trace_read()
+        o, lse = sa.fwd(q, k, v, alpha, beta=beta, **kw)
+        torch.cuda.synchronize()
+        names = set(sa.trace_read())
+        sa.trace_enable(False)
+    finally:
+        sa.select_forward(0)
+    assert ("fwd_tc" if kernel == 2 else "fwd_fast") in names, names
+    o_ref, lse_ref = oracle_fwd(q, k, v, alpha, beta=to_np(beta), **kw)
+    check_fwd(o, lse, o_ref, lse_ref, torch.bfloat16, f"prior forward kernel {kernel}")
 
 
 @pytest.mark.gpu
