@@ -216,7 +216,8 @@ sa_status sparse_attn_bwd_prior(const sa_params* p, const void* q, const void* k
  *   o        : device [L][B][H][D], dtype p->dtype                     (written)
  *   lse      : device fp32 [L][B][H] or NULL                           (written)
  * Any dtype and head dim of sparse_attn_fwd; no workspace.  Returns
- * SA_ERR_INVALID_ARG for pos outside [0, p->T).
+ * SA_ERR_INVALID_ARG for pos outside [0, p->T) and SA_ERR_UNSUPPORTED for a
+ * window above 256.
  */
 sa_status sparse_attn_decode(const sa_params* p, int32_t pos, const void* q, const void* k,
                              const void* v, const float* alpha, void* o, float* lse,

@@ -357,6 +357,7 @@ sa_status sparse_attn_decode_prior(const sa_params* p, int32_t pos, const void* 
   sa_status s = build_problem(p, &pb);
   if (s != SA_OK) return s;
   if (pos < 0 || pos >= pb.T) return SA_ERR_INVALID_ARG;
+  if (!sa::decode_supported(pb)) return SA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !alpha || !o) return SA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (lse && !aligned4(lse)) || !aligned4(alpha) || (beta && !aligned4(beta)))

@@ -241,6 +241,8 @@ cudaError_t launch_t(const DecArgs& a, long long units, cudaStream_t st) {
 
 }  // namespace
 
+bool decode_supported(const Problem& pb) { return pb.W <= 256; }
+
 cudaError_t launch_decode(const Problem& pb, int pos, const void* q, const void* k, const void* v,
                           const float* alpha, const float2* rope, void* o, float* lse,
                           cudaStream_t st, const float* beta) {

@@ -127,6 +127,8 @@ cudaError_t launch_alpha_from_theta(int L, const float* theta, float* alpha, cud
 cudaError_t launch_dtheta(int L, const float* theta, const float* dalpha, float* dtheta,
                           cudaStream_t st);
 // Single-token decode (sa_decode.cu): pb.T is the cache length, pos < pb.T.
+// Whether the decode kernel takes this problem (its member list fits shared memory).
+bool decode_supported(const Problem& pb);
 // beta: the new queries' log-prior on their offset members [units], or nullptr.
 cudaError_t launch_decode(const Problem& pb, int pos, const void* q, const void* k, const void* v,
                           const float* alpha, const float2* rope, void* o, float* lse,

@@ -95,6 +95,15 @@ def test_decode_equals_the_forward_row_for_the_last_position():
     assert (lse_d - lse_f[:, :, :, T - 1]).abs().max().item() <= 1e-5
 
 
+def test_decode_rejects_windows_it_cannot_hold():
+    import ctypes
+    p = sa.make_params((1, 1, 1, 1024, 64), torch.bfloat16, window=257)
+    dummy = ctypes.c_void_p(1 << 20)     # never dereferenced: validation comes first
+    st = sa.lib().sparse_attn_decode(ctypes.byref(p), 600, dummy, dummy, dummy, dummy, dummy,
+                                     None, None)
+    assert st == sa.SA_ERR_UNSUPPORTED
+
+
 def test_decode_rejects_positions_outside_the_cache():
     import ctypes
     p = sa.make_params((1, 1, 1, 64, 64), torch.bfloat16, window=12)
