@@ -6,12 +6,17 @@
 // interpolation with RoPE before the gather); the page measures inference
 // latency for exactly this gather (Results, efficiency).
 //
-// One warp per (layer, batch, head).  Scores: lanes take members in turn; a
-// member's key row (two rows for an interpolated offset) is loaded, rotated
-// at its own position and dotted with the rotated query held in shared
-// memory.  Softmax: warp reductions.  Output: lanes take head dims, walking
-// the members in order with their weights.  Only the W + S + 2 * n_offsets
-// rows a query attends are read from the cache.
+// One CTA of 128 threads per (layer, batch, head), so that a step is a few
+// dependent memory rounds deep (a single-token step is latency-bound):
+//   1. the member table, an L2 prefetch of every row it names, and the
+//      rotated, scaled query;
+//   2. scores, four threads per member, each a quarter of the head dims: the
+//      key row(s) (two rows for an interpolated offset, loaded together)
+//      rotated at their own positions and dotted with the query;
+//   3. a block-wide softmax;
+//   4. the output: the four warps take every fourth member, lanes take head
+//      dims, and the warps' partial sums meet in shared memory.
+// Only the W + S + 2 * n_offsets rows a query attends are read from the cache.
 #include "sa_device.cuh"
 #include "sa_internal.h"
 
@@ -19,11 +24,11 @@ namespace sa {
 
 namespace {
 
-constexpr int kDecWarps = 4;
+constexpr int kDecThreads = 128;                 // one CTA (4 warps) per unit
+constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kDecMaxMembers = 256 + SA_MAX_SINKS + SA_MAX_OFFSETS;
 
 struct DecArgs {
-  long long units;
   int B, H, Tc, W, n_off, S, pos;
   float scale;
   int f[SA_MAX_OFFSETS];
@@ -33,23 +38,34 @@ struct DecArgs {
   const float* beta;                   // log-prior on the offset members [units], or nullptr
 };
 
-// q_hat . RoPE(K[row]) over D dims; q_hat in shared memory.
+// Quarter `part` (0..3) of q_hat . (wa RoPE(K[ra]) + wb RoPE(K[rb])): the
+// rotation pairs [part * D/8, (part + 1) * D/8) of both rows (rb < 0: one
+// row), whose loads are all issued before any is used.
 template <typename T, int D>
-__device__ __forceinline__ float key_dot(const T* K, const float2* rope, int row, const float* qh) {
-  constexpr int HALF = D / 2, N = (HALF < 8 ? HALF : 8);
-  float acc = 0.f;
+__device__ __forceinline__ float member_score_part(const T* K, const float2* rope, int ra, int rb,
+                                                   float wa, float wb, const float* qh,
+                                                   int part) {
+  constexpr int HALF = D / 2, P = D / 8;
+  const int j0 = part * P;
+  const bool two = rb >= 0;
+  const int rb_ = two ? rb : ra;
+  float a1[P], a2[P], b1[P], b2[P];
+  float2 ca[P], cb[P];
+  load_row<T, P>(K + (size_t)ra * D + j0, a1);
+  load_row<T, P>(K + (size_t)ra * D + HALF + j0, a2);
+  load_cs<P>(rope + (size_t)ra * HALF + j0, ca);
+  load_row<T, P>(K + (size_t)rb_ * D + j0, b1);
+  load_row<T, P>(K + (size_t)rb_ * D + HALF + j0, b2);
+  load_cs<P>(rope + (size_t)rb_ * HALF + j0, cb);
+  rope_fwd<P>(a1, a2, ca);
+  rope_fwd<P>(b1, b2, cb);
+  float acc_a = 0.f, acc_b = 0.f;
 #pragma unroll
-  for (int j0 = 0; j0 < HALF; j0 += N) {
-    float x1[N], x2[N];
-    float2 cs[N];
-    load_row<T, N>(K + (size_t)row * D + j0, x1);
-    load_row<T, N>(K + (size_t)row * D + HALF + j0, x2);
-    load_cs<N>(rope + (size_t)row * HALF + j0, cs);
-    rope_fwd<N>(x1, x2, cs);
-#pragma unroll
-    for (int h = 0; h < N; ++h) acc += qh[j0 + h] * x1[h] + qh[HALF + j0 + h] * x2[h];
+  for (int h = 0; h < P; ++h) {
+    acc_a += qh[j0 + h] * a1[h] + qh[HALF + j0 + h] * a2[h];
+    acc_b += qh[j0 + h] * b1[h] + qh[HALF + j0 + h] * b2[h];
   }
-  return acc;
+  return two ? wa * acc_a + wb * acc_b : wa * acc_a;
 }
 
 template <typename T>
@@ -70,143 +86,139 @@ __device__ __forceinline__ void store_elt<__nv_bfloat16>(__nv_bfloat16* p, float
   *p = __float2bfloat16_rn(x);
 }
 
+// Block-wide reduction of one value per thread (max or sum); every thread
+// gets the result.
+template <bool MAX>
+__device__ __forceinline__ float block_reduce(float x, float* s_red) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const float y = __shfl_xor_sync(0xffffffffu, x, off);
+    x = MAX ? fmaxf(x, y) : x + y;
+  }
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = x;
+  __syncthreads();
+  float r = s_red[0];
+#pragma unroll
+  for (int w = 1; w < kDecWarps; ++w) r = MAX ? fmaxf(r, s_red[w]) : r + s_red[w];
+  __syncthreads();
+  return r;
+}
+
 template <typename T, int D>
-__global__ void __launch_bounds__(kDecWarps * 32) k_decode(const DecArgs a) {
-  __shared__ float s_q[kDecWarps][D];
-  __shared__ float s_w[kDecWarps][kDecMaxMembers];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long unit = (long long)blockIdx.x * kDecWarps + warp;
-  if (unit >= a.units) return;           // warps are independent (warp-level sync only)
-  const int layer = (int)(unit / (a.B * a.H));
+__global__ void __launch_bounds__(kDecThreads) k_decode(const DecArgs a) {
+  __shared__ float s_q[D];
+  __shared__ float s_p[kDecMaxMembers];          // scores, then unnormalised weights
+  __shared__ int s_ra[kDecMaxMembers], s_rb[kDecMaxMembers];   // rows (ra < 0: absent)
+  __shared__ float s_wa[kDecMaxMembers], s_wb[kDecMaxMembers];
+  __shared__ float s_o[kDecWarps][D];            // per-warp partial outputs
+  __shared__ float s_red[kDecWarps];
+  __shared__ OffGeo sg[SA_MAX_OFFSETS];
+  const int unit = blockIdx.x, t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int layer = unit / (a.B * a.H);
   const int W = a.W, S = a.S, n_off = a.n_off, pos = a.pos, Tc = a.Tc;
+  const int n = W + S + n_off;
   const T* Q = reinterpret_cast<const T*>(a.q) + (size_t)unit * D;
   const T* K = reinterpret_cast<const T*>(a.k) + (size_t)unit * Tc * D;
   const T* V = reinterpret_cast<const T*>(a.v) + (size_t)unit * Tc * D;
   T* O = reinterpret_cast<T*>(a.o) + (size_t)unit * D;
-  float* sw = s_w[warp];
-  float* sq = s_q[warp];
 
-  // offset geometry: lane k holds offset k
-  OffGeo og{};
   int bad = 0;
-  if (lane < n_off) {
-    og = offset_geometry(__ldg(a.alpha + layer), a.f[lane]);
-    bad = !og.ok;
+  if (t < n_off) {
+    sg[t] = offset_geometry(__ldg(a.alpha + layer), a.f[t]);
+    bad = !sg[t].ok;
   }
-  bad = __any_sync(0xffffffffu, bad);
-  if (bad) {
-    for (int d = lane; d < D; d += 32) store_elt<T>(O + d, __int_as_float(0x7fc00000));
-    if (lane == 0 && a.lse) a.lse[unit] = __int_as_float(0x7fc00000);
+  if (__syncthreads_or(bad)) {     // an offset with no defined row: NaN outputs
+    for (int d = t; d < D; d += kDecThreads) store_elt<T>(O + d, __int_as_float(0x7fc00000));
+    if (t == 0 && a.lse) a.lse[unit] = __int_as_float(0x7fc00000);
     return;
   }
 
-  // Prefetch into L2 every cache row the query reads (K and V of the window,
-  // the sinks and both rows of each offset): the rows are scattered over the
-  // cache, and the dependent steps below then find them in L2.
-  {
-    constexpr int kLines = (D * (int)sizeof(T) + 127) / 128;
-    auto prefetch_row = [&](int row) {
-#pragma unroll
-      for (int ln = 0; ln < kLines; ++ln) {
-        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(K + (size_t)row * D + ln * 128 / sizeof(T)));
-        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(V + (size_t)row * D + ln * 128 / sizeof(T)));
+  // member table (window lag m, sink m - W, offset m - W - S) and an L2
+  // prefetch of every K and V row it names; the rotated, scaled query
+  constexpr int kLines = (D * (int)sizeof(T) + 127) / 128;
+  for (int m = t; m < n; m += kDecThreads) {
+    int ra = -1, rb = -1;
+    float wa = 1.f, wb = 0.f;
+    if (m < W) {
+      if (pos - m >= 0) ra = pos - m;
+    } else if (m < W + S) {
+      if (m - W <= pos) ra = m - W;
+    } else {
+      const OffGeo g = sg[m - W - S];
+      if (pos - g.c >= 0) {
+        ra = pos - g.lo;
+        wa = g.wa;
+        if (g.w != 0.f) { rb = pos - g.lo - 1; wb = g.w; }
       }
-    };
-    for (int m = lane; m < W + S; m += 32) {
-      const int row = m < W ? pos - m : m - W;
-      if (row >= 0 && row <= pos) prefetch_row(row);
     }
-    if (lane < n_off && pos - og.c >= 0) {
-      prefetch_row(pos - og.lo);
-      if (og.w != 0.f) prefetch_row(pos - og.lo - 1);
+    s_ra[m] = ra; s_rb[m] = rb; s_wa[m] = wa; s_wb[m] = wb;
+#pragma unroll
+    for (int ln = 0; ln < kLines; ++ln) {
+      if (ra >= 0) {
+        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(K + (size_t)ra * D + ln * 128 / sizeof(T)));
+        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(V + (size_t)ra * D + ln * 128 / sizeof(T)));
+      }
+      if (rb >= 0) {
+        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(K + (size_t)rb * D + ln * 128 / sizeof(T)));
+        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(V + (size_t)rb * D + ln * 128 / sizeof(T)));
+      }
     }
   }
-
-  // rotated, scaled query at position pos
-  for (int j = lane; j < D / 2; j += 32) {
+  for (int j = t; j < D / 2; j += kDecThreads) {
     const float x1 = load_elt<T>(Q + j), x2 = load_elt<T>(Q + D / 2 + j);
     const float2 cs = __ldg(a.rope + (size_t)pos * (D / 2) + j);
-    sq[j] = (x1 * cs.x - x2 * cs.y) * a.scale;
-    sq[D / 2 + j] = (x2 * cs.x + x1 * cs.y) * a.scale;
+    s_q[j] = (x1 * cs.x - x2 * cs.y) * a.scale;
+    s_q[D / 2 + j] = (x2 * cs.x + x1 * cs.y) * a.scale;
   }
-  __syncwarp();
+  __syncthreads();
 
-  // scores of every member (window lags, sinks, offsets); invalid ones -inf
-  const int n = W + S + n_off;
-  float mx = -INFINITY;
-  for (int m = lane; m < n; m += 32) {
-    float s = -INFINITY;
-    if (m < W) {
-      const int row = pos - m;
-      if (row >= 0) s = key_dot<T, D>(K, a.rope, row, sq);
-    } else if (m < W + S) {
-      const int row = m - W;
-      if (row <= pos) s = key_dot<T, D>(K, a.rope, row, sq);
-    }
-    sw[m] = s;
-  }
-  // offsets: lane k's geometry, so the offset members go by lane; each
-  // carries the query's log-prior (0 without one)
+  // scores, four threads per member (a quarter of the dims each, summed by
+  // two shuffles); offset members carry the query's log-prior
   const float prior = a.beta ? __ldg(a.beta + unit) : 0.f;
-  for (int k0 = 0; k0 < n_off; k0 += 32) {
-    const int k = k0 + lane;
-    if (k < n_off) {
-      float s = -INFINITY;
-      if (pos - og.c >= 0) {
-        s = og.wa * key_dot<T, D>(K, a.rope, pos - og.lo, sq);
-        if (og.w != 0.f) s += og.w * key_dot<T, D>(K, a.rope, pos - og.lo - 1, sq);
-        s += prior;
-      }
-      sw[W + S + k] = s;
+  float mx = -INFINITY;
+  for (int m0 = 0; m0 < n; m0 += kDecThreads / 4) {     // uniform over the block
+    const int m = m0 + (t >> 2), part = t & 3;
+    const int ra = m < n ? s_ra[m] : -1;
+    float s = ra >= 0 ? member_score_part<T, D>(K, a.rope, ra, s_rb[m], s_wa[m], s_wb[m], s_q,
+                                                part)
+                      : 0.f;
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    if (m < n && part == 0) {
+      s = ra >= 0 ? s + (m >= W + S ? prior : 0.f) : -INFINITY;
+      s_p[m] = s;
+      mx = fmaxf(mx, s);
     }
   }
-  __syncwarp();
-  for (int m = lane; m < n; m += 32) mx = fmaxf(mx, sw[m]);
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  mx = block_reduce<true>(mx, s_red);
   float l = 0.f;
-  for (int m = lane; m < n; m += 32) {
-    const float e = sw[m] == -INFINITY ? 0.f : __expf(sw[m] - mx);
-    sw[m] = e;
+  for (int m = t; m < n; m += kDecThreads) {
+    const float e = s_p[m] == -INFINITY ? 0.f : __expf(s_p[m] - mx);
+    s_p[m] = e;
     l += e;
   }
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-  __syncwarp();
-  if (lane == 0 && a.lse) a.lse[unit] = mx + __logf(l);
-  const float inv = 1.f / l;
+  l = block_reduce<false>(l, s_red);     // (its barriers also publish s_p)
+  if (t == 0 && a.lse) a.lse[unit] = mx + __logf(l);
 
-  // output: lanes take dims d = lane, lane + 32, ...; members go in chunks
-  // of kChunk whose loads are all issued before any is consumed (the loop is
-  // bound by load latency, not arithmetic).  Member m's rows: window lag
-  // pos - m, sink m - W, offset rows pos - lo (weight 1 - w) and
-  // pos - lo - 1 (weight w).
+  // output: warp w takes members w, w + 4, ...; lanes take dims lane,
+  // lane + 32, ...; the loads of up to kChunk members are issued together
   constexpr int DPL = (D + 31) / 32;
   constexpr int kChunk = 8;
   float o[DPL];
 #pragma unroll
   for (int u = 0; u < DPL; ++u) o[u] = 0.f;
-  for (int m0 = 0; m0 < n; m0 += kChunk) {
+  for (int m0 = warp; m0 < n; m0 += kDecWarps * kChunk) {
     int ra[kChunk], rb[kChunk];
-    float wa[kChunk], wb[kChunk];
+    float pa[kChunk], pb[kChunk];
 #pragma unroll
     for (int j = 0; j < kChunk; ++j) {
-      const int m = m0 + j;
-      const float p = m < n ? sw[m] : 0.f;
-      ra[j] = 0; rb[j] = 0; wa[j] = 0.f; wb[j] = 0.f;
-      if (m < W + S) {
-        ra[j] = m < W ? max(pos - m, 0) : min(m - W, pos);
-        wa[j] = p;
-      } else {
-        const int k = min(m - W - S, n_off - 1);
-        const int lo = __shfl_sync(0xffffffffu, og.lo, k & 31);
-        const float w = __shfl_sync(0xffffffffu, og.w, k & 31);
-        const float ww = __shfl_sync(0xffffffffu, og.wa, k & 31);
-        if (p != 0.f) {
-          ra[j] = pos - lo; wa[j] = p * ww;
-          if (w != 0.f) { rb[j] = pos - lo - 1; wb[j] = p * w; }
-        }
-      }
+      const int m = m0 + j * kDecWarps;
+      const bool in = m < n && s_ra[m] >= 0;
+      const float p = in ? s_p[m] : 0.f;
+      ra[j] = in ? s_ra[m] : 0;
+      rb[j] = in && s_rb[m] >= 0 ? s_rb[m] : ra[j];
+      pa[j] = p * (in ? s_wa[m] : 0.f);
+      pb[j] = in && s_rb[m] >= 0 ? p * s_wb[m] : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < DPL; ++u) {
@@ -219,22 +231,29 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_decode(const DecArgs a) {
           xb[j] = load_elt<T>(V + (size_t)rb[j] * D + d);
         }
 #pragma unroll
-        for (int j = 0; j < kChunk; ++j) o[u] += wa[j] * xa[j] + wb[j] * xb[j];
+        for (int j = 0; j < kChunk; ++j) o[u] += pa[j] * xa[j] + pb[j] * xb[j];
       }
     }
   }
 #pragma unroll
   for (int u = 0; u < DPL; ++u) {
     const int d = lane + 32 * u;
-    if (d < D) store_elt<T>(O + d, o[u] * inv);
+    if (d < D) s_o[warp][d] = o[u];
+  }
+  __syncthreads();
+  const float inv = 1.f / l;
+  for (int d = t; d < D; d += kDecThreads) {
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) acc += s_o[w][d];
+    store_elt<T>(O + d, acc * inv);
   }
 }
 
 template <typename T, int D>
 cudaError_t launch_t(const DecArgs& a, long long units, cudaStream_t st) {
-  const unsigned grid = (unsigned)((units + kDecWarps - 1) / kDecWarps);
   trace_mark("decode", st, true);
-  k_decode<T, D><<<grid, kDecWarps * 32, 0, st>>>(a);
+  k_decode<T, D><<<(unsigned)units, kDecThreads, 0, st>>>(a);
   trace_mark("decode", st, false);
   return cudaGetLastError();
 }
@@ -253,7 +272,6 @@ cudaError_t launch_decode(const Problem& pb, int pos, const void* q, const void*
   a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.rope = rope; a.o = o; a.lse = lse;
   a.beta = beta;
   const long long units = pb.units();
-  a.units = units;
   const bool f32 = pb.dtype == SA_DTYPE_F32;
   switch (pb.D) {
     case 16: return f32 ? launch_t<float, 16>(a, units, st) : launch_t<__nv_bfloat16, 16>(a, units, st);
