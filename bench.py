@@ -68,14 +68,14 @@ def decode_bytes_per_token_head(wl, elt):
 # were taken on; a changed source reports null.
 MEASURED_TRAFFIC = {
     # profiles/staged_kernels_learned_train.md (one launch, 1048576 token-heads)
-    "learned_train/bwd_q_fast@8e3175152815": 779.8,
+    "learned_train/bwd_q_fast@6a730910219c": 779.8,
     # profiles/forward_and_decode_traffic.md
-    "pi_gate_train/bwd_q_fast@8e3175152815": 545.2,
-    "paper_fwd/fwd_fast@8e3175152815": 494.5,
-    "extrap_4x/fwd_fast@8e3175152815": 496.7,
-    "pi_skip/fwd_fast@8e3175152815": 491.7,
-    "long_sinks/fwd_tc@8e3175152815": 508.8,
-    "decode_4k/decode@8e3175152815": 8140.8,
+    "pi_gate_train/bwd_q_fast@6a730910219c": 545.4,
+    "paper_fwd/fwd_fast@6a730910219c": 494.5,
+    "extrap_4x/fwd_fast@6a730910219c": 496.4,
+    "pi_skip/fwd_fast@6a730910219c": 492.7,
+    "long_sinks/fwd_tc@6a730910219c": 509.0,
+    "decode_4k/decode@6a730910219c": 8121.8,
 }
 
 
