@@ -298,8 +298,10 @@ void sparse_attn_force_general(int on);
 
 /*
  * Diagnostics: which bf16 / D = 64 forward kernel sparse_attn_fwd runs.
- * 0 (default): the faster for the configuration (tensor-core for windows of
- * 32 or more, else CUDA-core); 1: the CUDA-core staged kernel; 2: the
+ * 0 (default): the faster for the configuration, as measured on B200: the
+ * tensor-core kernel for windows of 32 or more, except where its shared
+ * memory would leave it one CTA per SM while the CUDA-core kernel keeps two;
+ * otherwise the CUDA-core kernel.  1: the CUDA-core staged kernel; 2: the
  * tensor-core kernel where it applies (at most 16 sinks).  Other values mean
  * 0.  Process wide; sparse_attn_force_general takes precedence.
  */
