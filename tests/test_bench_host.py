@@ -1,0 +1,58 @@
+"""Host-side pieces of bench.py (no GPU): the byte accounting behind the
+roofline, the workload description in the JSON line, and the measured-traffic
+table's keys."""
+import re
+
+import bench
+from structured_sparse_attention_fibonacci_b200.inputs import WORKLOADS
+
+
+def test_algorithmic_bytes_per_token_head():
+    # forward: Q, K, V read and O written (4 rows of 64 bf16), LSE 4 B
+    assert bench.alg_bytes_per_token_head("fwd_fast", 64, 2) == 4 * 128 + 4
+    assert bench.alg_bytes_per_token_head("fwd_tc", 64, 2) == 516
+    # the saving forward also writes its context; the prior adds its 4 B
+    assert bench.alg_bytes_per_token_head("fwd_fast", 64, 2, context=296) == 812
+    assert bench.alg_bytes_per_token_head("fwd_fast", 64, 2, prior=True) == 520
+    # query and key sides: six rows and two fp32 values each
+    assert bench.alg_bytes_per_token_head("bwd_q_fast", 64, 2) == 6 * 128 + 8
+    assert bench.alg_bytes_per_token_head("bwd_q_fast", 64, 2, prior=True) == 784
+    assert bench.alg_bytes_per_token_head("bwd_kv_fast", 64, 2) == 776
+    # the RoPE pre-pass reads a row and writes it rotated; reductions count 0
+    assert bench.alg_bytes_per_token_head("rope_keys", 64, 2) == 256
+    assert bench.alg_bytes_per_token_head("reduce_dalpha", 64, 2) == 0
+
+
+def test_decode_bytes_count_every_member_row():
+    wl = WORKLOADS["decode_4k"]
+    rows = wl.window + wl.sinks + 2 * len(wl.offsets)          # 12 + 0 + 30
+    assert bench.decode_bytes_per_token_head(wl, 2) == 2 * 128 + 4 + 2 * rows * 128 == 11012
+
+
+def test_workload_config_names_the_workload():
+    for name, wl in WORKLOADS.items():
+        cfg = bench.workload_config(wl, 1)
+        assert cfg["workload"] == name
+        assert (cfg["L"], cfg["B"], cfg["H"], cfg["T"], cfg["D"]) == (wl.L, wl.B, wl.H, wl.T, wl.D)
+        assert cfg["parallelism"] == "replicas1" and cfg["global_batch"] == wl.B
+        assert ("prior" in cfg) == wl.prior
+        assert ("launch" in cfg) == wl.decode
+    assert bench.workload_config(WORKLOADS["learned_train"], 4)["global_batch"] == 32
+
+
+def test_measured_traffic_keys_name_workload_kernel_and_source_hash():
+    for key, per_unit in bench.MEASURED_TRAFFIC.items():
+        m = re.fullmatch(r"([a-z0-9_]+)/([a-z_]+)@([0-9a-f]{12})", key)
+        assert m, key
+        assert m.group(1) in WORKLOADS, key
+        assert per_unit > 0
+    # one capture campaign: every entry was taken on the same sources (a
+    # source change makes the bench report null until they are re-measured)
+    hashes = {k.split("@")[1] for k in bench.MEASURED_TRAFFIC}
+    assert len(hashes) <= 1
+    assert re.fullmatch(r"[0-9a-f]{12}", bench.kernel_source_hash())
+
+
+def test_aggregate_throughput_is_whole_job_units_per_second():
+    # 1048576 token-heads per rank, 4 ranks, 20 steps in 40 ms
+    assert bench.aggregate_throughput(1048576, 4, 20, 40.0) == 1048576 * 4 * 20 / 0.040
