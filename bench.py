@@ -175,6 +175,18 @@ def aggregate_throughput(units_per_rank, world, steps, ms_max):
 
 
 # ---- CPU baseline: the oracle as it stands, on a bounded sample -------------
+def cpu_model():
+    """The host CPU's model name (Linux), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def oracle_sample(wl, budget_s):
     """Time the fp32 oracle (forward, plus backward for training workloads) on
     as many whole layers (all their (batch, head) units, OpenMP-parallel) as
@@ -196,7 +208,7 @@ def oracle_sample(wl, budget_s):
             reps += 1
         cores = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
         units = wl.L * wl.B * wl.H
-        return {"value": reps * units / t, "unit": UNIT, "cores": cores, "kind": "oracle",
+        return {"value": reps * units / t, "unit": UNIT, "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
                 "sample": f"{reps} decode steps of {units} (layer, batch, head) units at "
                           f"position {wl.T - 1}, fp32 oracle", "seconds": round(t, 3)}
 
@@ -223,7 +235,7 @@ def oracle_sample(wl, budget_s):
     sample = (f"{n} of {wl.L} layers = {units} (layer, batch, head) units "
               f"({units * wl.T} token-heads), fp32 oracle "
               f"{'forward+backward' if wl.backward else 'forward'}")
-    return {"value": units * wl.T / t, "unit": UNIT, "cores": cores, "kind": "oracle",
+    return {"value": units * wl.T / t, "unit": UNIT, "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
             "sample": sample, "seconds": round(t, 3)}
 
 
