@@ -210,7 +210,7 @@ def oracle_sample(wl, budget_s):
         units = wl.L * wl.B * wl.H
         return {"value": reps * units / t, "unit": UNIT, "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
                 "sample": f"{reps} decode steps of {units} (layer, batch, head) units at "
-                          f"position {wl.T - 1}, fp32 oracle", "seconds": round(t, 3)}
+                          f"position {wl.T - 1}, fp32 oracle", "seconds": t}
 
     def one_layer(l):
         ts = make_inputs(wl, layers=range(l, l + 1))
@@ -236,7 +236,7 @@ def oracle_sample(wl, budget_s):
               f"({units * wl.T} token-heads), fp32 oracle "
               f"{'forward+backward' if wl.backward else 'forward'}")
     return {"value": units * wl.T / t, "unit": UNIT, "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
-            "sample": sample, "seconds": round(t, 3)}
+            "sample": sample, "seconds": t}
 
 
 def run_reference(args, rank, world):
@@ -250,7 +250,8 @@ def run_reference(args, rank, world):
         oracle_sample(wl, per_step_budget)
     vals = [oracle_sample(wl, per_step_budget) for _ in range(args.steps)]
     secs = sum(v["seconds"] for v in vals)
-    value = sum(v["value"] * v["seconds"] for v in vals) / secs
+    # time-weighted mean of the steps' rates (all units over all seconds)
+    value = sum(v["value"] * v["seconds"] for v in vals) / max(secs, 1e-12)
     cb = dict(vals[-1])
     cb["value"] = value
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,

@@ -56,3 +56,27 @@ def test_measured_traffic_keys_name_workload_kernel_and_source_hash():
 def test_aggregate_throughput_is_whole_job_units_per_second():
     # 1048576 token-heads per rank, 4 ranks, 20 steps in 40 ms
     assert bench.aggregate_throughput(1048576, 4, 20, 40.0) == 1048576 * 4 * 20 / 0.040
+
+
+def test_reference_arm_prints_one_json_line():
+    """`bench.py --impl reference` (the CPU oracle) on the tiny workload: one
+    JSON line with the contract's keys."""
+    import json
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(here, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny_fp32", "--steps", "2", "--warmup", "3"],
+                         capture_output=True, text=True, timeout=300, cwd=here)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 2
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
