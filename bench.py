@@ -187,7 +187,23 @@ def cpu_model():
     return None
 
 
-def oracle_sample(wl, budget_s):
+def on_one_thread(fn):
+    """fn()'s result with the oracle's OpenMP limited to one thread (None if
+    the OpenMP runtime cannot be reached)."""
+    import ctypes
+    try:
+        gomp = ctypes.CDLL("libgomp.so.1")
+    except OSError:
+        return None
+    before = gomp.omp_get_max_threads()
+    gomp.omp_set_num_threads(1)
+    try:
+        return fn()
+    finally:
+        gomp.omp_set_num_threads(before)
+
+
+def oracle_sample(wl, budget_s, single_thread=False):
     """Time the fp32 oracle (forward, plus backward for training workloads) on
     as many whole layers (all their (batch, head) units, OpenMP-parallel) as
     fit the time budget; at least one layer."""
@@ -231,12 +247,16 @@ def oracle_sample(wl, budget_s):
         t += one_layer(n)
         n += 1
     cores = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+    extra = {}
+    if single_thread:
+        # the same oracle on one thread, layer 0 only
+        extra["single_thread_layer0_s"] = on_one_thread(lambda: one_layer(0))
     units = n * wl.B * wl.H
     sample = (f"{n} of {wl.L} layers = {units} (layer, batch, head) units "
               f"({units * wl.T} token-heads), fp32 oracle "
               f"{'forward+backward' if wl.backward else 'forward'}")
     return {"value": units * wl.T / t, "unit": UNIT, "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
-            "sample": sample, "seconds": t}
+            "sample": sample, "seconds": t, **extra}
 
 
 def run_reference(args, rank, world):
@@ -465,7 +485,7 @@ def run_ours(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_sample(wl, args.cpu_budget_s)
+        cpu = oracle_sample(wl, args.cpu_budget_s, single_thread=True)
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -607,7 +627,7 @@ def run_ours_decode(args, rank, world, local_rank):
            "ms_per_step": e2e_ms / args.steps}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_sample(wl, args.cpu_budget_s)
+        cpu = oracle_sample(wl, args.cpu_budget_s, single_thread=True)
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
