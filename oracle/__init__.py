@@ -54,7 +54,7 @@ class Oracle:
             fwd.argtypes = head + [P] * 7
             bwd = getattr(lib, "oracle_bwd" + suffix)
             bwd.restype = ctypes.c_int
-            bwd.argtypes = head + [P] * 10
+            bwd.argtypes = head + [P] * 11
             geo = getattr(lib, "oracle_geometry" + suffix)
             geo.restype = ctypes.c_int
             geo.argtypes = [ctypes.c_float, ctypes.c_int32, ctypes.POINTER(ctypes.c_int64),
@@ -107,9 +107,11 @@ class Oracle:
         return (o, lse, p) if want_probs else (o, lse)
 
     def bwd(self, q, k, v, dout, alpha, *, window, offsets=FIB15, sinks=0,
-            rope_base=10000.0, scale=0.0, precision="f64", beta=None):
+            rope_base=10000.0, scale=0.0, precision="f64", beta=None, dalpha_units=False):
         """Backward for upstream dO: returns (dQ, dK, dV, dalpha[L]), and with
-        a log-prior beta [L, B, H, T] also dbeta: (dQ, dK, dV, dalpha, dbeta)."""
+        a log-prior beta [L, B, H, T] also dbeta: (dQ, dK, dV, dalpha, dbeta).
+        With dalpha_units=True one more element follows: each (layer, batch,
+        head) unit's share of dalpha, [L, B, H] (dalpha[l] is their sum)."""
         dt, ct = _np_dtype(precision)
         q, k, v, dout = (_prep(x, dt) for x in (q, k, v, dout))
         L, B, H, T, D = q.shape
@@ -120,16 +122,19 @@ class Oracle:
         dal = np.empty((L,), dtype=dt)
         bt = _prep(beta, dt).reshape(L, B, H, T) if beta is not None else None
         dbt = np.empty((L, B, H, T), dtype=dt) if beta is not None else None
+        dun = np.empty((L, B, H), dtype=dt) if dalpha_units else None
         fn = getattr(self.lib, "oracle_bwd_" + precision)
         rc = fn(L, B, H, T, D, int(window), len(offs), _ptr(offs, ctypes.c_int32), int(sinks),
                 float(rope_base), float(scale), _ptr(al, ctypes.c_float),
                 _ptr(q, ct), _ptr(k, ct), _ptr(v, ct), _ptr(dout, ct),
                 _ptr(dq, ct), _ptr(dk, ct), _ptr(dv, ct), _ptr(dal, ct),
                 _ptr(bt, ct) if bt is not None else None,
-                _ptr(dbt, ct) if dbt is not None else None)
+                _ptr(dbt, ct) if dbt is not None else None,
+                _ptr(dun, ct) if dun is not None else None)
         if rc != 0:
             raise ValueError(f"oracle_bwd rejected its arguments (rc={rc})")
-        return (dq, dk, dv, dal, dbt) if beta is not None else (dq, dk, dv, dal)
+        out = (dq, dk, dv, dal, dbt) if beta is not None else (dq, dk, dv, dal)
+        return out + (dun,) if dalpha_units else out
 
     def decode(self, q1, k, v, alpha, pos, *, window, offsets=FIB15, sinks=0,
                rope_base=10000.0, scale=0.0, precision="f64", beta=None):

@@ -271,13 +271,15 @@ int FN(oracle_fwd)(int L, int B, int H, int T, int D, int W, int n_off,
  * interpolation exists so that gradients reach alpha).  floor() is held fixed
  * (the right derivative at integer d); a second row i-lo-1 < 0 contributes 0.
  * beta (may be NULL): the forward's log-prior; dbeta (may be NULL) receives
- * its gradient [L][B][H][T].
+ * its gradient [L][B][H][T].  dalpha_units (may be NULL) receives each
+ * (layer, batch, head) unit's own share of dalpha, [L][B][H]: the terms that
+ * dalpha[l] sums in fixed order.
  */
 int FN(oracle_bwd)(int L, int B, int H, int T, int D, int W, int n_off,
                    const int32_t* offsets, int S, double rope_base, double scale,
                    const float* alpha, const real* Q, const real* K, const real* V,
                    const real* dO, real* dQ, real* dK, real* dV, real* dalpha,
-                   const real* beta, real* dbeta) {
+                   const real* beta, real* dbeta, real* dalpha_units) {
   prob_t p = {L, B, H, T, D, W, n_off, S, rope_base, scale, offsets, alpha};
   if (check(&p)) return -1;
   const double s = scale > 0 ? scale : 1.0 / sqrt((double)D);
@@ -387,6 +389,8 @@ int FN(oracle_bwd)(int L, int B, int H, int T, int D, int W, int n_off,
     for (int64_t r = 0; r < (int64_t)B * H; ++r) acc += dal_unit[(int64_t)l * B * H + r];
     dalpha[l] = acc;
   }
+  if (dalpha_units)
+    for (int64_t u = 0; u < units; ++u) dalpha_units[u] = dal_unit[u];
   free(dal_unit);
   return err ? -2 : 0;
 }

@@ -257,17 +257,25 @@ def pin_fd_inputs(orc):
 
 
 def pin_fd_alpha(orc):
+    """dalpha per layer, and each (layer, batch, head) unit's share of it,
+    against central finite differences of sum(dO * O) (the unit's share: of
+    that unit's part of the sum alone)."""
     q, k, v, do = _fd_problem()
-    _, _, _, dal = orc.bwd(q, k, v, do, FD_ALPHA, **FD_KW)
+    _, _, _, dal, dun = orc.bwd(q, k, v, do, FD_ALPHA, dalpha_units=True, **FD_KW)
     for l in range(2):
         for h in (3e-4,):
             ap, am = FD_ALPHA.copy(), FD_ALPHA.copy()
             ap[l] = np.float32(FD_ALPHA[l] + h)
             am[l] = np.float32(FD_ALPHA[l] - h)
-            lp = float((orc.fwd(q, k, v, ap, **FD_KW)[0] * do).sum())
-            lm = float((orc.fwd(q, k, v, am, **FD_KW)[0] * do).sum())
-            fd = (lp - lm) / (float(ap[l]) - float(am[l]))
+            op = orc.fwd(q, k, v, ap, **FD_KW)[0] * do
+            om = orc.fwd(q, k, v, am, **FD_KW)[0] * do
+            da = float(ap[l]) - float(am[l])
+            fd = (float(op.sum()) - float(om.sum())) / da
             assert abs(fd - dal[l]) <= 2e-3 * abs(fd) + 1e-6, (l, fd, dal[l])
+            for b in range(q.shape[1]):
+                for hh in range(q.shape[2]):
+                    fu = (float(op[l, b, hh].sum()) - float(om[l, b, hh].sum())) / da
+                    assert abs(fu - dun[l, b, hh]) <= 2e-3 * abs(fu) + 1e-6, (l, b, hh, fu)
 
 
 # -- learned-alpha map ---------------------------------------------------------
