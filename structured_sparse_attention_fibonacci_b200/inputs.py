@@ -19,6 +19,9 @@ from typing import Optional, Tuple
 import torch
 
 FIB15 = (1, 2, 3, 5, 8, 13, 21, 34, 55, 89, 144, 233, 377, 610, 987)
+# The power-of-2 base at the 4x evaluation length: every power of two below
+# 4096 (the control ladder, which reaches 1024 and 2048 there).
+POW2_4096 = tuple(1 << k for k in range(12))
 
 
 def alpha_linear_stagger(L: int = 16):
@@ -89,6 +92,12 @@ WORKLOADS = {
     "learned_train": Workload("learned_train", 16, 8, 8, 1024, 64, 12, 0, torch.bfloat16,
                               "learned", 4100, backward=True,
                               note="16 layers B=8 H=8 T=1024 d=64 bf16, W=12, learned alpha, fwd+bwd"),
+    "pow2_extrap": Workload("pow2_extrap", 16, 2, 8, 4096, 64, 12, 0, torch.bfloat16, "linear",
+                            9000, offsets=POW2_4096,
+                            note="the power-of-2 control base at the 4x evaluation length: "
+                                 "offsets 1, 2, 4, ..., 2048 with the linear stagger (reach "
+                                 "1.5 x 2048 = 3072 rows), 16 layers B=2 H=8 T=4096 d=64 bf16, "
+                                 "W=12"),
     "long_sinks": Workload("long_sinks", 1, 1, 16, 32768, 64, 64, 4, torch.bfloat16, "fixed", 5000,
                            note="B=1 H=16 T=32768 d=64 bf16, W=64, 4 sinks, alpha=1"),
     "pi_skip": Workload("pi_skip", 16, 8, 8, 1024, 64, 5, 0, torch.bfloat16, "fixed", 7000,

@@ -56,6 +56,12 @@ def test_workloads_take_the_pages_settings():
         assert WORKLOADS[name].window == g["best_window"][0]
     assert WORKLOADS["paper_fwd"].T == WORKLOADS["learned_train"].T == g["train_len"][0]
     assert WORKLOADS["extrap_4x"].T == g["eval_len"][0]
+    # the power-of-2 control at the evaluation length, with the linear stagger
+    p2 = WORKLOADS["pow2_extrap"]
+    assert p2.T == g["eval_len"][0] and p2.offsets == tuple(g["pow2_eval_ladder"])
+    assert max(p2.offsets) < p2.T <= 2 * max(p2.offsets)
+    assert p2.alpha_kind == "linear" and p2.window == g["best_window"][0]
+    assert p2.L == g["layers"][0] and p2.H * p2.D == g["hidden"][0]
     # the autoregressive periodic skip: the k previous keys plus the current
     # one, and one offset pi at alpha = 1
     for name in ("pi_skip", "pi_gate_train"):

@@ -7,8 +7,8 @@ import pytest
 import torch
 
 import structured_sparse_attention_fibonacci_b200 as sa
-from structured_sparse_attention_fibonacci_b200.inputs import (FIB15, WORKLOADS, make_dout,
-                                                                make_inputs)
+from structured_sparse_attention_fibonacci_b200.inputs import (FIB15, POW2_4096, WORKLOADS,
+                                                                make_dout, make_inputs)
 from parity import (check_bwd, check_dalpha, check_fwd, half_ulp_bf16, oracle_bwd, oracle_fwd,
                     run_gpu_fwd, to_np)
 
@@ -23,6 +23,13 @@ def _inputs(shape, dtype, seed, with_dout=True):
           for _ in range(4 if with_dout else 3)]
     return [t.to(DEV) for t in ts]
 
+
+# The largest offset table the library takes (32 entries): the Fibonacci and
+# power-of-2 ladders together, unsorted, with duplicates (1, 2 and 8 appear in
+# both), and entries whose distance at alpha = 1.5 exceeds T = 4096 (3000).
+OFF32 = (2048, 1, 3000, 2, 3, 5, 8, 13, 100, 21, 34, 55, 89, 144, 233, 377, 610, 987, 1, 2, 4,
+         8, 16, 32, 64, 128, 256, 512, 1024, 50, 7, 11)
+assert len(OFF32) == 32
 
 # (name, dtype, (L, B, H, T, D), window, sinks, alphas, offsets)
 SMALL = [
@@ -41,6 +48,11 @@ SMALL = [
     ("offsets_beyond_t_fp32", torch.float32, (1, 1, 1, 40, 64), 2, 0, [1.5], FIB15),
     ("custom_pow2_bf16", torch.bfloat16, (1, 1, 2, 260, 64), 8, 0, [1.0],
      (1, 2, 4, 8, 16, 32, 64, 128, 256)),
+    # the power-of-2 ladder at the 4x evaluation length: offsets up to 2048,
+    # reaching 3072 + 1 rows back at alpha = 1.5
+    ("pow2_ladder_t4096_bf16", torch.bfloat16, (2, 1, 1, 4096, 64), 12, 0, [1.0, 1.5], POW2_4096),
+    ("offsets32_t4096_bf16", torch.bfloat16, (1, 1, 1, 4096, 64), 12, 2, [1.5], OFF32),
+    ("offsets32_fp32", torch.float32, (1, 1, 1, 700, 32), 5, 1, [0.77], OFF32),
 ]
 
 
@@ -102,32 +114,47 @@ def _sample_units(wl, n):
     return sorted(units)
 
 
-@pytest.mark.parametrize("name", [n for n in WORKLOADS if not WORKLOADS[n].decode])
-def test_full_workload_sampled(name):
+FULL = [(n, "plain") for n in WORKLOADS if not WORKLOADS[n].decode] + \
+    [(n, "training") for n in WORKLOADS if WORKLOADS[n].backward and not WORKLOADS[n].prior]
+
+
+@pytest.mark.parametrize("name,mode", FULL, ids=[f"{n}-{m}" for n, m in FULL])
+def test_full_workload_sampled(name, mode):
+    """Every non-decode workload at full size.  "plain": sparse_attn_fwd /
+    sparse_attn_bwd.  "training": the launch the benchmark times for a
+    training workload -- the forward saving its context into a buffer, then
+    the backward reading it (with the forward's LSE).  O, LSE, dQ, dK, dV are
+    compared on sampled (layer, batch, head) units; dalpha on every layer."""
     wl = WORKLOADS[name]
     ts = make_inputs(wl, device=DEV)
     q, k, v = ts[:3]
     alpha = wl.alpha().to(DEV)
     kw = dict(window=wl.window, sinks=wl.sinks, offsets=wl.offsets, rope_base=wl.rope_base)
-    o, lse = run_gpu_fwd(q, k, v, alpha, **kw)
+    ctx = None
+    if mode == "training":
+        ctx = torch.full((sa.context_size(tuple(q.shape), q.dtype, **kw),), 0xFF,
+                         dtype=torch.uint8, device=DEV)
+    o, lse = sa.fwd(q, k, v, alpha, context=ctx, **kw)
+    torch.cuda.synchronize()
     for (l, b, h) in _sample_units(wl, 4):
         sl = (slice(l, l + 1), slice(b, b + 1), slice(h, h + 1))
         o_ref, lse_ref = oracle_fwd(q[sl], k[sl], v[sl], alpha[l:l + 1], **kw)
-        check_fwd(o[sl], lse[sl], o_ref, lse_ref, wl.dtype, f"{name} unit {(l, b, h)}")
+        check_fwd(o[sl], lse[sl], o_ref, lse_ref, wl.dtype, f"{name} {mode} unit {(l, b, h)}")
     if not wl.backward:
         return
     do = ts[3]
-    grads = sa.bwd(q, k, v, o, lse, do, alpha, **kw)
+    grads = sa.bwd(q, k, v, o, lse, do, alpha, context=ctx, **kw)
     torch.cuda.synchronize()
+    assert sa.device_error() == 0
     for (l, b, h) in _sample_units(wl, 3):
         sl = (slice(l, l + 1), slice(b, b + 1), slice(h, h + 1))
         ref = oracle_bwd(q[sl], k[sl], v[sl], do[sl], alpha[l:l + 1], **kw)
-        # d alpha of a single unit is not the layer sum: compare dQ/dK/dV here
+        # one unit's dalpha is not the layer sum: compare dQ/dK/dV here
         g = tuple(x[sl] for x in grads[:3]) + (torch.tensor(ref[3]),)
-        check_bwd(g, ref, wl.dtype, f"{name} bwd unit {(l, b, h)}")
-    # d alpha: every layer (each layer's value sums all its units)
+        check_bwd(g, ref, wl.dtype, f"{name} {mode} bwd unit {(l, b, h)}")
+    # dalpha: every layer, each against its own per-layer bound
     ref = oracle_bwd(q, k, v, do, alpha, **kw)
-    check_dalpha(grads[3], ref[3], wl.dtype, f"{name} dalpha")
+    check_dalpha(grads[3], ref[3], wl.dtype, f"{name} {mode} dalpha", units=ref.units)
 
 
 # ---- the staged bf16 d=64 forward and the general kernels on the same inputs ----
@@ -143,6 +170,9 @@ FAST = [
     ("fast_w7_odd", (2, 1, 1, 300, 64), 7, 3, [0.61, 1.44], FIB15),
     ("fast_long_1500", (1, 1, 1, 1700, 64), 12, 0, [1.5], FIB15),
     ("fast_pi_skip", (2, 1, 2, 300, 64), 5, 0, [1.0, 1.0], (16,)),
+    ("fast_pow2_t4096", (2, 1, 1, 4096, 64), 12, 0, [1.0, 1.5], POW2_4096),
+    ("fast_off32_t4096", (1, 1, 1, 4096, 64), 12, 2, [1.5], OFF32),
+    ("fast_off32_w64", (1, 1, 1, 2000, 64), 64, 4, [1.0], OFF32),
 ]
 
 
@@ -306,3 +336,59 @@ def test_tensors_beyond_2_31_elements():
     mid = H // 2
     for t in (o, dq, dk, dv):
         assert t[0, 0, mid].float().abs().max().item() == 0.0
+
+
+# ---- input magnitude: Q and K scaled up --------------------------------------
+# Scores grow with the square of the scale; a peaked softmax turns a score's
+# rounding into an output error.  The staged kernels round the rotated keys to
+# fp16 (2^-12 relative, reading 18), which keeps O within its bound up to about
+# x2 (measured on B200: x2 at 0.82 of the bound, x4 at 1.3x on the CUDA-core
+# kernel); the general kernels (fp32 throughout) keep the forward within it at
+# x100 and x10000, where only the fp32 LSE's relative rounding grows.
+
+def _scaled_inputs(shape, c, seed):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    q, k, v, do = (torch.randn(shape, generator=g, dtype=torch.float32) for _ in range(4))
+    return [t.to(torch.bfloat16).to(DEV) for t in (q * c, k * c, v, do)]
+
+
+@pytest.mark.parametrize("kernel", [1, 2], ids=["cuda_core", "tensor_core"])
+def test_staged_path_at_twice_the_input_scale(kernel):
+    shape = (2, 1, 2, 600, 64)
+    q, k, v, do = _scaled_inputs(shape, 2.0, seed=505)
+    alpha = torch.tensor([0.77, 1.23], device=DEV)
+    for W, S in ((12, 2), (64, 4)):
+        kw = dict(window=W, sinks=S)
+        sa.select_forward(kernel)
+        try:
+            o, lse = run_gpu_fwd(q, k, v, alpha, **kw)
+        finally:
+            sa.select_forward(0)
+        o_ref, lse_ref = oracle_fwd(q, k, v, alpha, **kw)
+        check_fwd(o, lse, o_ref, lse_ref, torch.bfloat16, f"x2 inputs W={W} (staged {kernel})")
+        if kernel == 1:
+            grads = sa.bwd(q, k, v, o, lse, do, alpha, **kw)
+            torch.cuda.synchronize()
+            check_bwd(grads, oracle_bwd(q, k, v, do, alpha, **kw), torch.bfloat16,
+                      f"x2 inputs W={W} backward")
+
+
+@pytest.mark.parametrize("c", [1e2, 1e4])
+def test_general_forward_at_large_input_scales(c):
+    shape = (1, 1, 2, 300, 64)
+    q, k, v, _ = _scaled_inputs(shape, c, seed=506)
+    alpha = torch.tensor([1.1234], device=DEV)
+    kw = dict(window=12, sinks=2)
+    sa.force_general(True)
+    try:
+        o, lse = run_gpu_fwd(q, k, v, alpha, **kw)
+    finally:
+        sa.force_general(False)
+    o_ref, lse_ref = oracle_fwd(q, k, v, alpha, **kw)
+    from parity import o_bound
+    err = np.abs(to_np(o) - o_ref) / o_bound(o_ref, torch.bfloat16)
+    assert err.max() <= 1.0, f"x{c:g} inputs: O err {err.max():.3f} x its bound"
+    # LSE of scores near c^2: each score is a 64-term fp32 dot product of
+    # c^2-sized products, rounded to about sqrt(64) * 2^-24 of itself
+    rel = np.abs(to_np(lse) - lse_ref) / np.maximum(np.abs(lse_ref), 1.0)
+    assert rel.max() <= 1e-5, f"x{c:g} inputs: LSE rel err {rel.max():.2e}"

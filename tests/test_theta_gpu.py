@@ -45,6 +45,10 @@ def test_learned_step_through_theta():
     dth = sa.dtheta(theta, dal)
     torch.cuda.synchronize()
     ref = oracle_bwd(q, k, v, do, alpha, window=12)
-    check_dalpha(dal, ref[3], torch.bfloat16, "dalpha at alpha(theta)")
+    check_dalpha(dal, ref[3], torch.bfloat16, "dalpha at alpha(theta)", units=ref.units)
     dth_ref = oracle.default().dtheta(to_np(theta), ref[3])
-    check_dalpha(dth, dth_ref, torch.bfloat16, "dtheta")
+    # each unit's share of dtheta: its dalpha share times the same chain-rule factor
+    th = to_np(theta)
+    sig = 1.0 / (1.0 + np.exp(-th))
+    units_th = ref.units * (sig * (1.0 - sig)).reshape(-1, 1, 1)
+    check_dalpha(dth, dth_ref, torch.bfloat16, "dtheta", units=units_th)
