@@ -11,8 +11,30 @@ T=1024, d=64, W=12, bf16, forward plus backward.  With N GPUs every rank runs
 its own batch (independent (layer, batch, head) units: weak scaling, no
 collective on the data path); the step time is the max over ranks.
 
-Prints one JSON line (rank 0).  See the design doc for the byte counts behind the
-roofline figures.
+Prints one JSON line (rank 0): the headline workload's throughput, its
+rooflines (HBM bytes and fp32 FMA work, by kernel and by phase), the end-to-end
+figure through host buffers, the CPU oracle baseline, and a "workloads" record
+timing the other benchmark configurations (forward only) the same way.
+
+Roofline bytes (per token-head, d = 64, bf16; the unique bytes the path must
+move, the definition the problem statement gives for the forward):
+  forward  : read Q, K, V, write O                       = 4 * 128       = 512 B
+  backward : read Q, K, V, O, dO and LSE, write dQ, dK, dV = 8 * 128 + 4  = 1028 B
+Per kernel, the backward's bytes are split as the kernels touch the tensors:
+the query side reads Q, K, V, dO, LSE and writes dQ (644 B); the key side
+writes dK and dV and carries O's read (384 B).  The RoPE pre-passes, the
+training context and the key-indexed weight blocks are intermediates the
+implementation chose, so they count 0.  The fp32 tiny case uses 4-byte
+elements.
+ALU work (per token-head): every distinct K/V row a query's members touch
+(window, sinks, both rows of each interpolated offset; rows shared by the
+window and an offset counted once) costs one D-long dot product and one
+D-long axpy in the forward (4 D FLOPs per row), and four in the backward
+with a saved context (dO.V, dq += g K, dK += g q, dV += p dO: 8 D FLOPs per
+row; a backward without context also recomputes the dot products, 10 D).
+The ALU peak is the fp32 FMA throughput measured in the same run by the
+library's probe (packed fp32x2 FMAs, register-only); the nominal figure is
+148 SMs x 128 lanes x 2 FLOPs per clock at the sampled SM clock.
 """
 import argparse
 import hashlib
@@ -29,29 +51,178 @@ sys.path.insert(0, HERE)
 METRIC = "sparse-attn fwd/bwd tokens·heads/s at T=1024/4096; HBM GB/s vs B200 peak"
 UNIT = "tokens·heads/s"
 FALLBACK_HBM_GBS = 6650.0
+B200_SMS, FP32_LANES_PER_SM = 148, 128
+# Configurations timed beside the headline in the "workloads" record: the
+# other four problem-statement configurations and the power-of-2 control.
+OTHER_WORKLOADS = ("tiny_fp32", "paper_fwd", "extrap_4x", "long_sinks", "pow2_extrap")
 
-# Algorithmic bytes per token-head for d=64 bf16 (2-byte elements, fp32 LSE / D):
-#   forward  : read Q, K, V; write O and LSE
-#   bwd query: read Q, K, V, O, dO, LSE; write dQ and D
-#   bwd key  : read Q, K, V, dO, LSE, D; write dK, dV
-#   RoPE pre-pass (rope_keys / rope_queries): read K (or Q), write it rotated
-# (the whole backward: Q, K, V, O, dO, dQ, dK, dV and LSE = 1028 B)
-def alg_bytes_per_token_head(kernel, D, elt, context=0, prior=False):
-    """Bytes a kernel must move per token-head: every input row read once and
-    every output written once.  ``context``: bytes per token-head the saving
-    forward also writes into the training context (0 without one); ``prior``:
-    the fp32 log-prior is read by the forward and the query side, which also
-    writes its gradient."""
+
+def alg_bytes_per_token_head(kernel, D, elt, prior=False):
+    """The roofline bytes a kernel is credited with per token-head (see the
+    module docstring): the forward kernels Q, K, V and O; the backward query
+    side Q, K, V, dO, LSE and dQ; the key side dK, dV and O; pre-passes 0.
+    With a log-prior the forward also reads beta and the query side reads
+    beta and writes dbeta (4 B each)."""
     row = D * elt
     if kernel.startswith("fwd"):
-        return 4 * row + 4 + context + (4 if prior else 0)
+        return 4 * row + (4 if prior else 0)
     if kernel.startswith("bwd_q"):
-        return 6 * row + 8 + (8 if prior else 0)
+        return 5 * row + 4 + (8 if prior else 0)
     if kernel.startswith("bwd_kv"):
-        return 6 * row + 8
-    if kernel.startswith("rope"):      # RoPE pre-pass: read a row, write it rotated
-        return 2 * row
+        return 3 * row
     return 0
+
+
+def phase_bytes_per_token_head(phase, D, elt, prior=False):
+    """forward: Q, K, V, O; backward: Q, K, V, O, dO, dQ, dK, dV and LSE
+    (plus beta, and dbeta in the backward, with a log-prior)."""
+    row = D * elt
+    if phase == "forward":
+        return 4 * row + (4 if prior else 0)
+    return 8 * row + 4 + (8 if prior else 0)
+
+
+def distinct_rows(alpha, offsets, window, sinks):
+    """Distinct K/V rows a query far from the sequence start touches at this
+    alpha: window lags 0..W-1, each offset's lags lo and (when w != 0) lo + 1,
+    the sinks.  d = fp32 product alpha * f, lo = floor(d)."""
+    import numpy as np
+    lags = set(range(window))
+    a32 = np.float32(alpha)
+    for f in offsets:
+        d = float(a32 * np.float32(f))
+        lo = int(np.floor(d))
+        lags.add(lo)
+        if d != lo:
+            lags.add(lo + 1)
+    return len(lags) + sinks
+
+
+def alg_flops(wl, phase, context=True):
+    """fp32 FLOPs of one pass over the workload (see the module docstring)."""
+    per_row = {"forward": 4, "backward": 8 if context else 10}[phase] * wl.D
+    rows = sum(distinct_rows(a, wl.offsets, wl.window, wl.sinks) for a in wl.alpha().tolist())
+    return per_row * rows * (wl.B * wl.H * wl.T)
+
+
+def kernel_flops(wl, kernel, context=True):
+    """fp32 FLOPs one launch of a kernel is credited with: the forward 4 D per
+    distinct row, the query side 4 D (6 D when it recomputes the dot products
+    without a context), the key side 4 D; pre-passes and reductions 0."""
+    if kernel.startswith("fwd"):
+        per = 4
+    elif kernel.startswith("bwd_q"):
+        per = 4 if context else 6
+    elif kernel.startswith("bwd_kv"):
+        per = 4
+    else:
+        return 0
+    rows = sum(distinct_rows(a, wl.offsets, wl.window, wl.sinks) for a in wl.alpha().tolist())
+    return per * wl.D * rows * (wl.B * wl.H * wl.T)
+
+
+def fma_peak(sa, torch, dev, reps=5):
+    """The ALU roofline's peak, measured now: the library's register-only fp32
+    FMA probe (scalar and packed), 8 CTAs of 256 threads per SM, best of
+    `reps` launches of each, timed with CUDA events on the current stream.
+    The nominal figure is 148 SMs x 128 lanes x 2 FLOPs at the GPU's maximum
+    SM clock."""
+    blocks, threads, iters = B200_SMS * 8, 256, 4096
+    out = torch.empty(blocks * threads, dtype=torch.float32, device=dev)
+    best = {}
+    for packed in (0, 1):
+        for _ in range(2):
+            sa.fma_probe(out, blocks, threads, iters, packed)
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            flops = sa.fma_probe(out, blocks, threads, iters, packed)
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        best["packed" if packed else "scalar"] = flops / (min(ts) / 1e3) / 1e12
+    try:
+        mhz = float(torch.cuda.get_device_properties(dev).clock_rate) / 1e3
+    except Exception:
+        mhz = None
+    if not mhz:
+        mhz = 1965.0
+    nominal = B200_SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+    kind = max(best, key=best.get)
+    return {"peak": best[kind], "source": f"measured in-run: fp32 FMA probe ({kind}), "
+                                          f"{blocks} CTAs x {threads} threads",
+            "probe_TFLOPs": best, "nominal": nominal, "nominal_clock_mhz": mhz}
+
+
+def time_forward_workload(sa, torch, dev, name, steps, warmup, peak, alu_peak):
+    """Device time of `steps` forward passes of a benchmark workload (its
+    inputs resident in HBM), with its rooflines; inputs smaller than L2 are
+    timed step by step with an L2 flush (a 256 MiB write) between steps."""
+    from structured_sparse_attention_fibonacci_b200.inputs import WORKLOADS, make_inputs
+    wl = WORKLOADS[name]
+    q, k, v = make_inputs(wl, device=str(dev))[:3]
+    alpha = wl.alpha().to(dev)
+    kw = dict(window=wl.window, sinks=wl.sinks, offsets=wl.offsets, rope_base=wl.rope_base)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:4], dtype=torch.float32, device=dev)
+    ws_n = sa.workspace_size(tuple(q.shape), q.dtype, backward=False, **kw)
+    ws = torch.empty(max(1, ws_n), dtype=torch.uint8, device=dev)
+    elt = q.element_size()
+    in_bytes = 3 * q.numel() * elt
+    small = in_bytes < 126 * 2 ** 20
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev) if small else None
+
+    def step():
+        sa.fwd(q, k, v, alpha, out=o, lse=lse, workspace=ws, **kw)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    launches = 0
+    if small:
+        total = 0.0
+        for _ in range(steps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            step()
+            b.record()
+            torch.cuda.synchronize()
+            launches += sa.last_launch_count()
+            total += a.elapsed_time(b)
+        ms = total / steps
+    else:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            step()
+            launches += sa.last_launch_count()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / steps
+    sa.trace_enable(True)
+    for _ in range(steps):
+        step()
+    tr = sa.trace_read()
+    sa.trace_enable(False)
+    kern = {n: t / c for n, (t, c) in tr.items()}
+    bpt = phase_bytes_per_token_head("forward", wl.D, elt, wl.prior)
+    fl = alg_flops(wl, "forward")
+    fwd_k = max(kern, key=kern.get)
+    gbs = bpt * wl.token_heads / (ms / 1e3) / 1e9
+    k_gbs = bpt * wl.token_heads / (kern[fwd_k] / 1e3) / 1e9
+    rec = {"config": wl.note, "ms_per_step": ms, "value": wl.token_heads / (ms / 1e3),
+           "unit": UNIT, "gpu_launches": launches, "l2": "flushed between steps (256 MiB write)"
+           if small else "inputs larger than L2",
+           "kernels_ms": kern, "alg_bytes_per_token_head": bpt,
+           "hbm": {"achieved_GBps": gbs, "frac": gbs / peak, "kernel": fwd_k,
+                   "kernel_frac": k_gbs / peak},
+           "alu": {"alg_flops": fl, "achieved_TFLOPs": fl / (ms / 1e3) / 1e12,
+                   "frac": fl / (ms / 1e3) / 1e12 / alu_peak if alu_peak else None}}
+    del q, k, v, o, lse, ws, flush
+    torch.cuda.empty_cache()
+    return rec
 
 
 def decode_bytes_per_token_head(wl, elt):
@@ -62,14 +233,12 @@ def decode_bytes_per_token_head(wl, elt):
     return 2 * row + 4 + 2 * rows * row
 
 
-# dram__bytes_read.sum + dram__bytes_write.sum per token-head (per
-# (layer, batch, head) for decode) from the ncu captures summarised under
-# profiles/, keyed by workload, kernel and the hash of the kernel sources they
-# were taken on; a changed source reports null.
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per token-head
+# (per (layer, batch, head) for decode) of the dominant kernel, from one ncu
+# capture per entry; keyed by workload, kernel and the hash of the kernel
+# sources the capture ran (kernel_source_hash): a changed source reports null.
 MEASURED_TRAFFIC = {
-    # profiles/staged_kernels_learned_train.md (one launch, 1048576 token-heads)
     "learned_train/bwd_q_fast@6a730910219c": 779.8,
-    # profiles/forward_and_decode_traffic.md
     "pi_gate_train/bwd_q_fast@6a730910219c": 545.4,
     "paper_fwd/fwd_fast@6a730910219c": 494.5,
     "extrap_4x/fwd_fast@6a730910219c": 496.4,
@@ -338,15 +507,20 @@ def run_ours(args, rank, world, local_rank):
         ctx = torch.empty(n_ctx, dtype=torch.uint8, device=dev) if n_ctx else None
     launches = [0]
 
-    def step():
+    def fwd_call():
         sa.fwd(q, k, v, alpha, out=o, lse=lse, context=ctx if wl.backward else None, beta=beta,
                **kw)
-        n = sa.last_launch_count()
+        launches[0] += sa.last_launch_count()
+
+    def bwd_call():
+        sa.bwd(q, k, v, o, lse, do, alpha, dq=dq, dk=dk, dv=dv, dalpha=dal, workspace=ws,
+               context=ctx, beta=beta, dbeta=dbeta, **kw)
+        launches[0] += sa.last_launch_count()
+
+    def step():
+        fwd_call()
         if wl.backward:
-            sa.bwd(q, k, v, o, lse, do, alpha, dq=dq, dk=dk, dv=dv, dalpha=dal, workspace=ws,
-                   context=ctx, beta=beta, dbeta=dbeta, **kw)
-            n += sa.last_launch_count()
-        launches[0] += n
+            bwd_call()
 
     def barrier():
         if world > 1:
@@ -382,32 +556,72 @@ def run_ours(args, rank, world, local_rank):
     ms_max = max_over_ranks(ms, dev)
     value = aggregate_throughput(wl.token_heads, world, args.steps, ms_max)
 
-    # per-kernel times of the same steps (library trace: events on the launch stream)
+    # per-kernel times of the same steps, forward and backward traced apart
+    # (library trace: CUDA events around each launch, on its stream)
+    phases = [("forward", fwd_call)] + ([("backward", bwd_call)] if wl.backward else [])
+    traced = {ph: {} for ph, _ in phases}
     sa.trace_enable(True)
     for _ in range(args.steps):
-        step()
-    torch.cuda.synchronize()
-    trace = sa.trace_read()
+        for ph, call in phases:
+            call()
+            for n, (t, c) in sa.trace_read().items():
+                tt, cc = traced[ph].get(n, (0.0, 0))
+                traced[ph][n] = (tt + t, cc + c)
     sa.trace_enable(False)
-    kernels = {n: {"ms_per_launch": t / c, "launches": c} for n, (t, c) in trace.items()}
-    dominant = max(kernels, key=lambda n: kernels[n]["ms_per_launch"] * kernels[n]["launches"])
     elt = 2 if wl.dtype == torch.bfloat16 else 4
     peak, peak_kind = measured_peaks()
-    # the training context per token-head: fp32 probabilities of every
-    # member, fp32 row-score differences per offset, the fp16 rotated query
-    ctx_th = ((wl.window + wl.sinks + 2 * len(wl.offsets)) * 4 + wl.D * 2) if wl.backward else 0
-    per_th = alg_bytes_per_token_head(dominant, wl.D, elt, ctx_th, wl.prior)
-    bytes_launch = per_th * wl.token_heads
-    achieved = bytes_launch / (kernels[dominant]["ms_per_launch"] / 1e3) / 1e9
-    key = f"{wl.name}/{dominant}@{kernel_source_hash()}"
-    traffic = MEASURED_TRAFFIC.get(key)
+    alu = fma_peak(sa, torch, dev)
+    context = bool(wl.backward and ctx is not None)
+    kernels = {}
+    for ph, _ in phases:
+        for n, (t, c) in traced[ph].items():
+            key = n if n not in kernels else f"{n} ({ph})"
+            ms_l = t / c
+            b = alg_bytes_per_token_head(n, wl.D, elt, wl.prior) * wl.token_heads
+            fl = kernel_flops(wl, n, context)
+            kernels[key] = {"phase": ph, "ms_per_launch": ms_l, "launches": c,
+                            "alg_GBps": b / (ms_l / 1e3) / 1e9 if b else None,
+                            "alg_TFLOPs": fl / (ms_l / 1e3) / 1e12 if fl else None}
+    dominant = max(kernels, key=lambda n: kernels[n]["ms_per_launch"] * kernels[n]["launches"])
+    dom = kernels[dominant]
+    bytes_launch = alg_bytes_per_token_head(dominant, wl.D, elt, wl.prior) * wl.token_heads
+    achieved = bytes_launch / (dom["ms_per_launch"] / 1e3) / 1e9
+    src_hash = kernel_source_hash()
+    traffic = MEASURED_TRAFFIC.get(f"{wl.name}/{dominant}@{src_hash}")
+    phase_ms = {ph: sum(kk["ms_per_launch"] * kk["launches"] for kk in kernels.values()
+                        if kk["phase"] == ph) / args.steps for ph, _ in phases}
+    phase_ms["step"] = sum(phase_ms.values())
+    ph_rec = {}
+    for ph, msp in phase_ms.items():
+        if ph == "step":
+            bpt = sum(phase_bytes_per_token_head(p, wl.D, elt, wl.prior) for p, _ in phases)
+            fl = sum(alg_flops(wl, p, context) for p, _ in phases)
+        else:
+            bpt = phase_bytes_per_token_head(ph, wl.D, elt, wl.prior)
+            fl = alg_flops(wl, ph, context)
+        gbs = bpt * wl.token_heads / (msp / 1e3) / 1e9
+        tfs = fl / (msp / 1e3) / 1e12
+        ph_rec[ph] = {"ms": msp, "alg_bytes_per_token_head": bpt, "achieved_GBps": gbs,
+                      "frac": gbs / peak, "alg_flops": fl, "achieved_TFLOPs": tfs,
+                      "alu_frac": tfs / alu["peak"] if alu["peak"] else None}
     roofline = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
                 "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                 "alg_bytes_per_launch": bytes_launch,
-                "traffic": traffic * wl.token_heads if traffic is not None else None}
-    for n, kk in kernels.items():
-        b = alg_bytes_per_token_head(n, wl.D, elt, ctx_th, wl.prior) * wl.token_heads
-        kk["alg_GBps"] = b / (kk["ms_per_launch"] / 1e3) / 1e9 if b else None
+                "traffic": traffic * wl.token_heads if traffic is not None else None,
+                "traffic_source": (f"ncu@{src_hash}" if traffic is not None else
+                                   f"none: no ncu capture of sources {src_hash}"),
+                "phases": {ph: {k_: r[k_] for k_ in ("ms", "alg_bytes_per_token_head",
+                                                     "achieved_GBps", "frac")}
+                           for ph, r in ph_rec.items()}}
+    dom_fl = kernel_flops(wl, dominant, context)
+    dom_tf = dom_fl / (dom["ms_per_launch"] / 1e3) / 1e12
+    roofline_alu = {"bound": "alu", "kernel": dominant, "achieved": dom_tf, "peak": alu["peak"],
+                    "peak_source": alu["source"], "peak_nominal": alu["nominal"],
+                    "unit": "TFLOP/s", "frac": dom_tf / alu["peak"] if alu["peak"] else None,
+                    "alg_flops_per_launch": dom_fl,
+                    "phases": {ph: {"ms": r["ms"], "alg_flops": r["alg_flops"],
+                                    "achieved_TFLOPs": r["achieved_TFLOPs"],
+                                    "frac": r["alu_frac"]} for ph, r in ph_rec.items()}}
 
     # End to end through the public API: every step copies its inputs in from
     # pinned host memory and its results back out.  Two device buffer sets
@@ -487,14 +701,31 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(wl, args.cpu_budget_s, single_thread=True)
 
+    # the other benchmark configurations, forward only, timed the same way
+    # (every rank runs them, so that all ranks take the same steps)
+    workloads = None
+    if not args.no_workloads:
+        del q, k, v, o, lse, host, sets
+        if wl.backward:
+            del dq, dk, dv, ws, ctx, do
+        torch.cuda.empty_cache()
+        workloads = {}
+        for name in OTHER_WORKLOADS:
+            if name != wl.name:
+                workloads[name] = time_forward_workload(sa, torch, dev, name, args.steps,
+                                                        args.warmup, peak, alu["peak"])
+
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32", "data": "synthetic",
                 "config": workload_config(wl, world), "roofline": roofline,
+                "roofline_alu": roofline_alu, "alu_peak": alu,
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches, "clocks": clocks,
                 "kernels": kernels, "kernel_source": kernel_source_hash()}
+        if workloads is not None:
+            line["workloads"] = workloads
         print(json.dumps(line), flush=True)
     return 0
 
@@ -583,13 +814,14 @@ def run_ours_decode(args, rank, world, local_rank):
     # a step is exactly one decode launch: its device time is the graph's
     # time per step (the traced launches above also hold the host's gaps)
     achieved = bytes_launch / (ms_max / args.steps / 1e3) / 1e9
+    src_hash = kernel_source_hash()
+    traffic = MEASURED_TRAFFIC.get(f"{wl.name}/decode@{src_hash}")
     roofline = {"bound": "hbm", "kernel": "decode", "achieved": achieved, "peak": peak,
                 "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                 "alg_bytes_per_launch": bytes_launch,
-                "traffic": None}
-    traffic = MEASURED_TRAFFIC.get(f"{wl.name}/decode@{kernel_source_hash()}")
-    if traffic is not None:
-        roofline["traffic"] = traffic * units
+                "traffic": traffic * units if traffic is not None else None,
+                "traffic_source": (f"ncu@{src_hash}" if traffic is not None else
+                                   f"none: no ncu capture of sources {src_hash}")}
 
     # end to end: the new token's q, k, v rows in, O and LSE out, every step
     kr_h = kc_h[:, :, :, pos].contiguous().pin_memory()
@@ -648,6 +880,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="learned_train")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the forward timings of the other configurations")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--reference-budget-s", type=float, default=120.0)
     args = ap.parse_args()

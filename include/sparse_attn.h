@@ -253,11 +253,15 @@ sa_status sparse_attn_dtheta(int32_t L, const float* theta, const float* dalpha,
  * entry point exists for callers that cannot let a library call cudaMalloc --
  * applications whose device memory belongs to a pooling allocator that must
  * account for every byte, and embedders or latency-critical services that
- * forbid allocation after start-up.  It computes exactly what sparse_attn_fwd
- * computes (same arguments minus the workspace), but keeps its only scratch,
- * the RoPE cos/sin table, in a fixed file-scope device array of
- * SA_NOALLOC_SCRATCH_BYTES (8 MiB) that every GPU loading this library holds
- * until the process exits.
+ * forbid allocation after start-up.  It computes what sparse_attn_fwd
+ * computes (same arguments minus the workspace), to within the same parity
+ * tolerances but not bit for bit: with no workspace for rotated keys, bf16 /
+ * D = 64 problems with windows up to 256 run the staged CUDA-core kernel with
+ * the keys rotated in shared memory (sparse_attn_fwd may choose the
+ * tensor-core kernel there), and all others the general kernels.  Its only
+ * scratch, the RoPE cos/sin table, lives in a fixed file-scope device array
+ * of SA_NOALLOC_SCRATCH_BYTES (8 MiB) that every GPU loading this library
+ * holds until the process exits.
  *   Limit: T * (D/2) * 8 bytes must fit in SA_NOALLOC_SCRATCH_BYTES (for D=64,
  *   T <= 32768); larger problems return SA_ERR_UNSUPPORTED before any work.
  *   Set-up: the first call on a device looks up the array's device address
@@ -275,12 +279,47 @@ sa_status sparse_attn_fwd_noalloc(const sa_params* p, const void* q, const void*
                                   void* stream);
 
 /*
- * Device error word of the staged kernels: bit 0 is set when a bounded wait
- * for a staging copy gave up (the kernel then left its outputs incomplete and
- * returned rather than wait without end).  Reading synchronises with the
+ * Device error word of the staged kernels.  Reading synchronises with the
  * device; with clear != 0 the word is reset.  Returns -1 on a CUDA error.
+ *   bit 0: a bounded wait for a staging copy gave up (the kernel then left
+ *          its outputs incomplete and returned rather than wait without end);
+ *   bit 1: a row index outside the rows staged in shared memory, or a staging
+ *          round larger than its ring -- checked only by the bounds-checking
+ *          build (compiled with SA_DEBUG_BOUNDS), which records and skips the
+ *          access;
+ *   bit 2: a finite input beyond the range of the staged 16-bit operands:
+ *          |RoPE(K)| / 256 (and, in the backward, |RoPE(Q)| * scale / 256)
+ *          above 65504, i.e. rotated key or scaled query elements beyond about
+ *          1.68e7; for the tensor-core forward also |RoPE(Q)| * scale above
+ *          65504.  Outputs of such a call are not valid.
  */
 int32_t sparse_attn_device_error(int clear);
+
+/*
+ * Diagnostics of the bounded waits (process wide, for tests):
+ * sparse_attn_set_wait_limit sets how many SM clocks a staging wait waits
+ * before it gives up (<= 0: the default, 1e9 clocks, about half a second).
+ * With sparse_attn_plant_stall(1), every CTA of later staged launches expects
+ * 16 bytes more in its first staging round than any copy delivers, so that
+ * round's wait runs out: bit 0 of the device error word is set and the kernel
+ * returns without finishing its outputs.  Nothing faults and nothing waits
+ * beyond the limit.  Off (0) by default.
+ */
+void sparse_attn_set_wait_limit(long long clocks);
+void sparse_attn_plant_stall(int on);
+
+/*
+ * Diagnostics: throughput probe of the fp32 FMA pipe, the peak of the ALU
+ * roofline of the CUDA-core kernels (the paper has no counterpart).  Launches
+ * `blocks` CTAs of `threads` threads (32..256, a multiple of 32); each thread
+ * runs 8 independent register-only FMA chains of `iters` steps, scalar
+ * fma.rn.f32 (packed = 0) or packed fma.rn.f32x2 (packed != 0), then writes one
+ * float to out[blocks * threads] (device).  FLOPs per launch:
+ * blocks * threads * iters * 8 * 2 * (packed ? 2 : 1).  The caller times it
+ * (CUDA events on `stream`).  Returns SA_ERR_INVALID_ARG for bad sizes.
+ */
+sa_status sparse_attn_diag_fma_probe(int32_t blocks, int32_t threads, int32_t iters,
+                                     int32_t packed, float* out, void* stream);
 
 /* Static, NUL-terminated description of a status code. */
 const char* sparse_attn_status_string(sa_status s);

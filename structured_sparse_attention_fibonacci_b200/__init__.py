@@ -22,7 +22,10 @@ import torch
 FIB15 = (1, 2, 3, 5, 8, 13, 21, 34, 55, 89, 144, 233, 377, 610, 987)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsparse_attn.so")
+# The library; SPARSE_ATTN_LIBRARY may name another build of the same sources
+# (build.py also writes libsparse_attn_bounds.so, the bounds-checking build).
+LIB_PATH = os.environ.get("SPARSE_ATTN_LIBRARY") or os.path.join(_HERE, "libsparse_attn.so")
+BOUNDS_LIB_PATH = os.path.join(_HERE, "libsparse_attn_bounds.so")
 
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE, SA_ERR_CUDA, SA_ERR_INTERNAL = range(6)
 SA_DTYPE_F32, SA_DTYPE_BF16 = 0, 1
@@ -35,7 +38,11 @@ EXPORTED = ("sparse_attn_fwd", "sparse_attn_bwd", "sparse_attn_workspace_size",
             "sparse_attn_fwd_noalloc", "sparse_attn_device_error", "sparse_attn_select_forward",
             "sparse_attn_context_size", "sparse_attn_fwd_train", "sparse_attn_bwd_ctx",
             "sparse_attn_decode", "sparse_attn_alpha_from_theta", "sparse_attn_dtheta",
-            "sparse_attn_fwd_prior", "sparse_attn_bwd_prior", "sparse_attn_decode_prior")
+            "sparse_attn_fwd_prior", "sparse_attn_bwd_prior", "sparse_attn_decode_prior",
+            "sparse_attn_set_wait_limit", "sparse_attn_plant_stall", "sparse_attn_diag_fma_probe")
+
+# Device error word bits (sparse_attn_device_error)
+ERR_WAIT, ERR_BOUNDS, ERR_RANGE = 1, 2, 4
 
 
 class SaParams(ctypes.Structure):
@@ -106,6 +113,13 @@ def lib():
         L.sparse_attn_select_forward.argtypes = [ctypes.c_int]
         L.sparse_attn_device_error.restype = ctypes.c_int32
         L.sparse_attn_device_error.argtypes = [ctypes.c_int]
+        L.sparse_attn_set_wait_limit.restype = None
+        L.sparse_attn_set_wait_limit.argtypes = [ctypes.c_longlong]
+        L.sparse_attn_plant_stall.restype = None
+        L.sparse_attn_plant_stall.argtypes = [ctypes.c_int]
+        L.sparse_attn_diag_fma_probe.restype = ctypes.c_int
+        L.sparse_attn_diag_fma_probe.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                 ctypes.c_int32, fp, vp]
         L.sparse_attn_trace_enable.restype = None
         L.sparse_attn_trace_enable.argtypes = [ctypes.c_int]
         L.sparse_attn_trace_read.restype = ctypes.c_int32
@@ -163,9 +177,34 @@ def select_forward(which: int = 0) -> None:
 
 
 def device_error(clear: bool = True) -> int:
-    """Device error word of the staged kernels (bit 0: a bounded staging wait
-    gave up); synchronises with the device; cleared after reading by default."""
+    """Device error word of the staged kernels (ERR_WAIT: a bounded staging
+    wait gave up; ERR_BOUNDS: a bounds violation seen by the bounds-checking
+    build; ERR_RANGE: an input beyond the staged operands' fp16 range);
+    synchronises with the device; cleared after reading by default."""
     return int(lib().sparse_attn_device_error(int(bool(clear))))
+
+
+def fma_probe(out, blocks, threads, iters, packed, stream=None) -> int:
+    """Diagnostics: launch the fp32 FMA throughput probe (see
+    sparse_attn_diag_fma_probe); out: a float32 CUDA tensor of blocks *
+    threads elements.  Returns the probe's FLOPs per launch."""
+    if out.dtype != torch.float32 or not out.is_cuda or out.numel() < blocks * threads:
+        raise ValueError("out must be a float32 CUDA tensor of blocks * threads elements")
+    _check("sparse_attn_diag_fma_probe",
+           lib().sparse_attn_diag_fma_probe(int(blocks), int(threads), int(iters), int(packed),
+                                            _ptr(out), _stream_handle(stream)))
+    return int(blocks) * int(threads) * int(iters) * 8 * 2 * (2 if packed else 1)
+
+
+def set_wait_limit(clocks: int = 0) -> None:
+    """Diagnostics: SM clocks a staging wait waits before giving up (0: default)."""
+    lib().sparse_attn_set_wait_limit(int(clocks))
+
+
+def plant_stall(on: bool = True) -> None:
+    """Diagnostics (failure-path test): later staged launches expect 16 bytes
+    in their first staging round that no copy delivers, so that wait gives up."""
+    lib().sparse_attn_plant_stall(int(bool(on)))
 
 
 def trace_enable(on: bool = True) -> None:
@@ -221,7 +260,8 @@ def _check_prior(shape, dev, **named):
 
 
 def fwd(q, k, v, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0, scale=0.0,
-        out=None, lse=None, want_lse=True, stream=None, context=None, beta=None):
+        out=None, lse=None, want_lse=True, stream=None, context=None, beta=None,
+        workspace=None):
     """Sparse attention forward over all layers: returns (O, LSE or None).
 
     q, k, v: CUDA tensors [L, B, H, T, D] (bf16 or fp32, contiguous).
@@ -230,6 +270,8 @@ def fwd(q, k, v, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0, sc
     runs as sparse_attn_fwd_train and saves what bwd(..., context=) reuses.
     beta: CUDA fp32 [L, B, H, T], a log-prior added to every offset member's
     score of each query (sparse_attn_fwd_prior).
+    workspace: an optional CUDA uint8 buffer of at least
+    workspace_size(..., backward=False) bytes (else one is allocated per call).
     """
     if beta is not None:
         return _fwd_prior(q, k, v, alpha, beta, window=window, offsets=offsets, sinks=sinks,
@@ -248,7 +290,12 @@ def fwd(q, k, v, alpha, *, window, offsets=FIB15, sinks=0, rope_base=10000.0, sc
                     rope_base=rope_base, scale=scale)
     L = lib()
     ws_n = int(L.sparse_attn_workspace_size(ctypes.byref(p), 0))
-    ws = torch.empty(ws_n, dtype=torch.uint8, device=dev) if ws_n else None
+    if workspace is not None:
+        if workspace.device != dev or workspace.numel() * workspace.element_size() < ws_n:
+            raise ValueError(f"workspace must be a CUDA buffer of at least {ws_n} bytes")
+        ws, ws_n = workspace, workspace.numel() * workspace.element_size()
+    else:
+        ws = torch.empty(ws_n, dtype=torch.uint8, device=dev) if ws_n else None
     st = L.sparse_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(out),
                            _ptr(lse), _ptr(ws), ws_n, _stream_handle(stream))
     _check("sparse_attn_fwd", st)

@@ -16,6 +16,8 @@ namespace {
 thread_local int32_t g_last_launches = 0;
 int g_force_general = 0;  // diagnostics: route every call through the general kernels
 int g_fwd_select = 0;     // diagnostics: 0 auto, 1 CUDA-core staged forward, 2 tensor-core forward
+long long g_wait_limit = 0;  // diagnostics: staging wait limit in SM clocks (0: default)
+int g_plant_stall = 0;       // diagnostics: failure-path test of the bounded waits
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -113,6 +115,8 @@ cudaError_t launch_fwd_dispatch(const Problem& pb, const FwdPtrs& a, cudaStream_
              : launch_fwd_general(pb, a, st, launches);
 }
 
+WaitCfg wait_cfg() { return WaitCfg{g_wait_limit, g_plant_stall}; }
+
 void trace_mark(const char* kernel, cudaStream_t st, bool begin) {
   std::lock_guard<std::mutex> lock(g_trace_mu);
   if (!g_trace_on) return;
@@ -151,6 +155,10 @@ void sparse_attn_force_general(int on) { g_force_general = on != 0; }
 
 void sparse_attn_select_forward(int which) { g_fwd_select = (which == 1 || which == 2) ? which : 0; }
 
+void sparse_attn_set_wait_limit(long long clocks) { g_wait_limit = clocks > 0 ? clocks : 0; }
+
+void sparse_attn_plant_stall(int on) { g_plant_stall = on != 0; }
+
 void sparse_attn_trace_enable(int on) {
   std::lock_guard<std::mutex> lock(g_trace_mu);
   g_trace_on = on != 0;
@@ -184,12 +192,13 @@ int32_t sparse_attn_trace_read(int32_t max, const char** names, double* total_ms
 }
 
 int32_t sparse_attn_device_error(int clear) {
-  unsigned fwd = 0, fwd_tc = 0, bwd = 0;
+  unsigned fwd = 0, fwd_tc = 0, bwd = 0, prep = 0;
   if (sa::fast_fwd_read_error(&fwd, clear != 0) != cudaSuccess ||
       sa::fast_fwd_tc_read_error(&fwd_tc, clear != 0) != cudaSuccess ||
-      sa::fast_bwd_read_error(&bwd, clear != 0) != cudaSuccess)
+      sa::fast_bwd_read_error(&bwd, clear != 0) != cudaSuccess ||
+      sa::prep_read_error(&prep, clear != 0) != cudaSuccess)
     return -1;
-  return (int32_t)(fwd | fwd_tc | bwd);
+  return (int32_t)(fwd | fwd_tc | bwd | prep);
 }
 
 size_t sparse_attn_workspace_size(const sa_params* p, int backward) {

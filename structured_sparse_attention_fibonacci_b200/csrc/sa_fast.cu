@@ -45,6 +45,8 @@ struct FastArgs {
   const float* alpha; const float2* rope;
   __nv_bfloat16* o; float* lse;
   unsigned* err;
+  long long wait_limit;                // bounded waits: SM clocks (0: the default)
+  int stall;                           // failure-path test: plant a stall in round 1
   float* save_p;                       // SAVE: [units][W+S+n_off][T] member probabilities
   float* save_dt;                      // SAVE: [units][n_off][T] row-score differences
   __half* save_q;                      // SAVE: [units][T][64] fp16 of RoPE(Q) * scale / 256
@@ -121,7 +123,7 @@ __device__ __forceinline__ int next_far(const int* s_kind, int k, int n_off) {
 // rows, so the fp32 recurrence stays within ~1e-6 of the table); odd runs
 // touch their two chunks in the opposite order (bank-conflict-free).
 __device__ __forceinline__ void rotate_rows(unsigned char* buf, int RB, const float2* rope, int a,
-                                            int b) {
+                                            int b, unsigned* err) {
   const int n = b - a;
   if (n <= 0) return;
   const int runs = blockDim.x >> 2;
@@ -158,6 +160,7 @@ __device__ __forceinline__ void rotate_rows(unsigned char* buf, int RB, const fl
       cs[h].y = cs[h].y * st[h].x + cs[h].x * st[h].y;
       cs[h].x = c2;
     }
+    if (half_overflow8(x1) | half_overflow8(x2)) atomicOr(err, kErrRange);
     const uint4 u1 = pack8_h(x1), u2 = pack8_h(x2);
     *c0 = par ? u2 : u1;
     *c1 = par ? u1 : u2;
@@ -180,8 +183,8 @@ __device__ __forceinline__ int stage_keys(Stager& s, unsigned char* ring, int RB
   if (S_stage) stage_plain(s, sinkb, K, min(a.S, T), a.S);
   if (stage_commit_wait(s)) { stage_drain(s); return 1; }
   if (!PRE) {
-    rotate_rows(ring, RB, a.rope, max(lo, 0), min(hi, T));
-    if (S_stage) rotate_rows(sinkb, 0, a.rope, 0, min(a.S, T));
+    rotate_rows(ring, RB, a.rope, max(lo, 0), min(hi, T), a.err);
+    if (S_stage) rotate_rows(sinkb, 0, a.rope, 0, min(a.S, T), a.err);
     __syncthreads();
   }
   return 0;
@@ -241,7 +244,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
     }
     return;
   }
-  Stager stg{&bar, 0u, a.err};
+  Stager stg = make_stager(&bar, a.err, a.wait_limit, a.stall);
 
   // This lane's slice of its 4 queries, rotated and scaled (times the inverse
   // of the key staging factor), first half = chunk c + 4 * par.
@@ -282,6 +285,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
         y0[h] = q[qq][h] * (kKeyStage * kKeyStage);
         y1[h] = q[qq][h + 8] * (kKeyStage * kKeyStage);
       }
+      if (half_overflow8(y0) | half_overflow8(y1)) atomicOr(a.err, kErrRange);
       uint4* dst = reinterpret_cast<uint4*>(a.save_q + ub + (size_t)i * kD);
       dst[h0] = pack8_h(y0);
       dst[h1] = pack8_h(y1);
@@ -298,6 +302,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
 
   // ---------------- pass 1: scores ----------------
   if (stage_keys<PRE>(stg, ring, RB, sinkb, a, K, 1, T, win_lo, win_hi)) return;
+  dbg_rows(stg, ig - W + 1, ig + 4);
   {
     int d0 = 0;
     // lags in blocks of 3 (the loop body's code stays small: measured on B200,
@@ -346,6 +351,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
       for (int m = kk; m < nx; m = next_far(s_kind, m, n_off)) {
         const OffGeo g = sg[m];
         const int two = SAVE || g.w != 0.f;
+        dbg_rows(stg, ig - g.lo - 1 + (two ? 0 : 1), ig - g.lo + 4);
         const unsigned char* p = ring + (size_t)((ig - g.lo - 1) & (RB - 1)) * kRowBytes + off0;
         float pa[4] = {0.f, 0.f, 0.f, 0.f}, pb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -438,6 +444,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
   stage_ring(stg, ring, RB, V, T, win_lo, win_hi);
   stage_plain(stg, sinkb, V, min(S, T), S);
   if (stage_commit_wait(stg)) { stage_drain(stg); return; }
+  dbg_rows(stg, ig - W + 1, ig + 4);
   {
     int d0 = 0;
     while (W - d0 >= 3) { window_pv<3>(ring, RB, ig, d0, off0, d1, grp_sc, a.sc_stride, o); d0 += 3; }
@@ -470,6 +477,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
       for (int m = kk; m < nx; m = next_far(s_kind, m, n_off)) {
         const OffGeo g = sg[m];
         const int two = g.w != 0.f;
+        dbg_rows(stg, ig - g.lo - 1 + (two ? 0 : 1), ig - g.lo + 4);
         float p[4];
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) p[qq] = grp_sc[qq * a.sc_stride + W + S + m];
@@ -505,7 +513,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_fast(const FastArgs a) {
   }
 }
 
-__device__ unsigned g_fwd_err;   // bit 0: a staging wait gave up
+__device__ unsigned g_fwd_err;   // error bits as listed in sa_stage.cuh
 
 int ring_rows_for(const Problem& pb) {
   int rr = 32;   // a power of two: ring slots are row & (rr - 1)
@@ -551,6 +559,9 @@ cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& p, void* keys_ws, 
   a.save_p = save_p; a.save_dt = save_dt; a.save_q = reinterpret_cast<__half*>(save_q);
   a.beta = p.beta;
   cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&a.err), g_fwd_err);
+  const WaitCfg wc = wait_cfg();
+  a.wait_limit = wc.limit;
+  a.stall = wc.stall;
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((long long)pb.units() * a.n_tiles);
   auto launch = [&](auto kernel) -> cudaError_t {

@@ -52,6 +52,8 @@ struct FastBwdArgs {
   float* dal_part;                       // [units][n_tiles]
   float* sink_k; float* sink_v;          // [units][n_tiles][S][64]
   unsigned* err;
+  long long wait_limit;                // bounded waits: SM clocks (0: the default)
+  int stall;                           // failure-path test: plant a stall in round 1
   const float* ctx_p;                    // training context: [units][W+S+n_off][T] probabilities
   const float* ctx_dt;                   // ... and [units][n_off][T] row-score differences
   const float* beta;                     // log-prior on offset members [units][T], or nullptr
@@ -189,6 +191,7 @@ __device__ __forceinline__ int member_dots(const FastBwdArgs& a, Stager& stg,
   stage_ring(stg, ring, RB, src, T, win_lo, win_hi);
   stage_plain(stg, sinkb, src, min(S, T), S);
   if (stage_commit_wait(stg)) { stage_drain(stg); return 1; }
+  dbg_rows(stg, ig - W + 1, ig + 4);
 #define SA_CALL(LC) window_dots<LC, F16>(ring, RB, ig, d0, off0, d1, c, x, val_row, i_own, mx)
   SA_WINDOW_CHUNKS(W, SA_CALL)
 #undef SA_CALL
@@ -230,6 +233,7 @@ __device__ __forceinline__ int member_dots(const FastBwdArgs& a, Stager& stg,
     }
     for (int kk = kb; kk < nx; kk = next_far(s_kind, kk, a.n_off)) {
       const OffGeo g = sg[kk];
+      dbg_rows(stg, ig - g.lo - 1, ig - g.lo + 4);
       const unsigned char* p = ring + (size_t)((ig - g.lo - 1) & (RB - 1)) * kRowBytes + off0;
       float pa[4], pb[4];
 #pragma unroll
@@ -320,7 +324,7 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
     if (t == 0) a.dal_part[(size_t)unit * a.n_tiles + tile] = qnan;
     return;
   }
-  Stager stg{&bar, 0u, a.err};
+  Stager stg = make_stager(&bar, a.err, a.wait_limit, a.stall);
   const int off0 = half0_off(c, par), d1 = half1_off(c, par) - off0;
   const int lr = 4 * gid + c;
   float* my_sc = sc + (size_t)lr * st;
@@ -433,10 +437,12 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
       // j + lo (row a) and j + lo + 1 (row b)
       const size_t tile_base = (size_t)unit * a.n_tiles;
       const size_t blk = (size_t)a.NS * M;
+      const size_t blk_end = (size_t)gridDim.x * blk;   // weight entries of the launch
       for (int d = 0; d < W; ++d) {
         const int j = i - d;
         if (j < 0) break;
         const size_t off = (tile_base + j / M) * blk + (size_t)d * M + (j % M);
+        dbg_check(a.err, off < blk_end);
         a.gblk[off] = __float2bfloat16_rn(my_sc[d]);
         a.pblk[off] = __float2bfloat16_rn(my_dp[d]);
       }
@@ -447,11 +453,13 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
         const int ja = i - g.lo, jb = i - g.lo - 1;
         if (ja >= 0) {
           const size_t off = (tile_base + ja / M) * blk + (size_t)(W + kk) * M + (ja % M);
+          dbg_check(a.err, off < blk_end);
           a.gblk[off] = __float2bfloat16_rn(g.wa * gg);
           a.pblk[off] = __float2bfloat16_rn(g.wa * pp);
         }
         if (jb >= 0) {
           const size_t off = (tile_base + jb / M) * blk + (size_t)(W + n_off + kk) * M + (jb % M);
+          dbg_check(a.err, off < blk_end);
           a.gblk[off] = __float2bfloat16_rn(g.w * gg);
           a.pblk[off] = __float2bfloat16_rn(g.w * pp);
         }
@@ -492,6 +500,7 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
     stage_ring(stg, ring, RB, Kh, T, win_lo, win_hi);
     stage_plain(stg, sinkb, Kh, min(S, T), S);
     if (stage_commit_wait(stg)) { stage_drain(stg); return; }
+    dbg_rows(stg, ig - W + 1, ig + 4);
 #define SA_CALL(LC) window_axpy<LC, true>(ring, RB, ig, d0, off0, d1, grp_sc, st, x)
     SA_WINDOW_CHUNKS(W, SA_CALL)
 #undef SA_CALL
@@ -523,6 +532,7 @@ __global__ void __launch_bounds__(kFastM) k_bwd_q_fast(const FastBwdArgs a) {
         float gq[4];
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq) gq[qq] = grp_sc[qq * st + W + S + kk];
+        dbg_rows(stg, ig - g.lo - 1 + (two ? 0 : 1), ig - g.lo + 4);
         const unsigned char* p = ring + (size_t)((ig - g.lo - 1) & (RB - 1)) * kRowBytes + off0;
 #pragma unroll
         for (int u = 0; u < 5; ++u) {
@@ -644,6 +654,7 @@ __device__ __forceinline__ int key_pass(const FastBwdArgs& a, Stager& stg, unsig
   stage_ring(stg, ring, RB, src, T, r0, high);
   stage_plain(stg, wblk, wsrc, 2 * a.NS, 2 * a.NS);     // NS * M bf16 = 2 NS rows of 128 B
   if (stage_commit_wait(stg)) { stage_drain(stg); return 1; }
+  dbg_rows(stg, rg, rg + W + 3);
   // window: key rg+kk takes query row rg+d0+u at lag d0 + u - kk
   int d0 = 0;
   while (d0 < W) {
@@ -700,6 +711,7 @@ __device__ __forceinline__ int key_pass(const FastBwdArgs& a, Stager& stg, unsig
         fa[0] = bf16lo(ua.x); fa[1] = bf16hi(ua.x); fa[2] = bf16lo(ua.y); fa[3] = bf16hi(ua.y);
         fb[0] = bf16lo(uv.x); fb[1] = bf16hi(uv.x); fb[2] = bf16lo(uv.y); fb[3] = bf16hi(uv.y);
       }
+      dbg_rows(stg, rg + g.lo, rg + g.lo + (two ? 5 : 4));
       const unsigned char* p = ring + (size_t)((rg + g.lo) & (RB - 1)) * kRowBytes + off0;
 #pragma unroll
       for (int u = 0; u < 5; ++u) {
@@ -757,7 +769,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_bwd_kv_fast(const FastBwdArgs a) 
     return;
   }
   (void)n_off;
-  Stager stg{&bar, 0u, a.err};
+  Stager stg = make_stager(&bar, a.err, a.wait_limit, a.stall);
   const int off0 = half0_off(c, par), d1 = half1_off(c, par) - off0;
   const int h0 = c + 4 * par, h1 = c + 4 - 4 * par;
   const size_t blk = ((size_t)unit * a.n_tiles + tile) * (size_t)a.NS * M;
@@ -827,7 +839,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_bwd_kv_fast(const FastBwdArgs a) 
   }
 }
 
-__device__ unsigned g_bwd_err;   // bit 0: a staging wait gave up
+__device__ unsigned g_bwd_err;   // error bits as listed in sa_stage.cuh
 
 struct FastBwdLayout {
   int ring_rows, sc_stride, NS, n_tiles;
@@ -918,6 +930,9 @@ cudaError_t launch_bwd_fast(const Problem& pb, const BwdPtrs& p, cudaStream_t st
   cudaError_t e;
   if ((e = cudaGetSymbolAddress(reinterpret_cast<void**>(&a.err), g_bwd_err)) != cudaSuccess)
     return e;
+  const WaitCfg wc = wait_cfg();
+  a.wait_limit = wc.limit;
+  a.stall = wc.stall;
   const long long n_rows = pb.units() * pb.T;
   if (!ctx && (e = launch_rope_rows(p.k, p.rope, pb.T, n_rows, kKeyStage, khat, st,
                                     "rope_keys")) != cudaSuccess)

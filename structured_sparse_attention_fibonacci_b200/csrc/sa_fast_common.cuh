@@ -47,21 +47,29 @@ __device__ __forceinline__ uint4 pack8_h(const float* x) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// Whether any of 8 finite values would overflow fp16 (|x| >= 65520 rounds to
+// infinity): the range limit of the 16-bit staged operands.
+__device__ __forceinline__ bool half_overflow8(const float* x) {
+  bool over = false;
+#pragma unroll
+  for (int h = 0; h < 8; ++h) over |= isfinite(x[h]) && fabsf(x[h]) >= 65520.f;
+  return over;
+}
+
 __device__ __forceinline__ uint4 pack8(const float* x) {
   return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
                     pack_bf16x2(x[6], x[7]));
 }
 
-// Dot product and axpy over a lane's 16 dims with packed fp32 FMAs
-// (two per instruction).
+// Dot product and axpy over a lane's 16 dims with packed fp32 FMAs (two per
+// instruction).  The dot product keeps one packed accumulator chain: measured
+// on B200 faster than two chains summed at the end (two more adds per call).
 __device__ __forceinline__ float dot16(const float (&q)[16], const float (&x)[16]) {
-  float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
+  float2 a = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int h = 0; h < 16; h += 4) {
+  for (int h = 0; h < 16; h += 2)
     a = __ffma2_rn(make_float2(q[h], q[h + 1]), make_float2(x[h], x[h + 1]), a);
-    b = __ffma2_rn(make_float2(q[h + 2], q[h + 3]), make_float2(x[h + 2], x[h + 3]), b);
-  }
-  return (a.x + b.x) + (a.y + b.y);
+  return a.x + a.y;
 }
 
 __device__ __forceinline__ void axpy16(float (&o)[16], float p, const float (&x)[16]) {

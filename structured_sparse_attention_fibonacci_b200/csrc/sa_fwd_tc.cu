@@ -47,6 +47,8 @@ struct TcFwdArgs {
   const float* alpha; const float2* rope;
   __nv_bfloat16* o; float* lse;
   unsigned* err;
+  long long wait_limit;                // bounded waits: SM clocks (0: the default)
+  int stall;                           // failure-path test: plant a stall in round 1
   const float* beta;                   // log-prior on offset members [units][T], or nullptr
 };
 
@@ -64,6 +66,7 @@ __device__ __forceinline__ int next_far(const int* s_kind, int k, int n_off) {
 __device__ __forceinline__ void q_frags(const TcFwdArgs& a, const __nv_bfloat16* Q, int qb,
                                         int lane, uint32_t (&aq)[4][4]) {
   const int g = lane >> 2, t = lane & 3;
+  bool over = false;                            // a value beyond fp16's range
 #pragma unroll
   for (int h = 0; h < 2; ++h) {                 // row g (regs 0, 2) and g + 8 (regs 1, 3)
     const int row = min(qb + g + 8 * h, a.T - 1);
@@ -78,11 +81,15 @@ __device__ __forceinline__ void q_frags(const TcFwdArgs& a, const __nv_bfloat16*
         const uint32_t hi2 = __ldg(reinterpret_cast<const unsigned*>(qr + d + 32));
         const float4 c = __ldg(reinterpret_cast<const float4*>(cs + d));
         const float x0 = bf16lo(lo2), x1 = bf16hi(lo2), y0 = bf16lo(hi2), y1 = bf16hi(hi2);
-        aq[ks][h + 2 * p] = pack_h2((x0 * c.x - y0 * c.y) * a.scale, (x1 * c.z - y1 * c.w) * a.scale);
-        aq[ks + 2][h + 2 * p] =
-            pack_h2((y0 * c.x + x0 * c.y) * a.scale, (y1 * c.z + x1 * c.w) * a.scale);
+        float r[8] = {(x0 * c.x - y0 * c.y) * a.scale, (x1 * c.z - y1 * c.w) * a.scale,
+                      (y0 * c.x + x0 * c.y) * a.scale, (y1 * c.z + x1 * c.w) * a.scale,
+                      0.f, 0.f, 0.f, 0.f};
+        over |= half_overflow8(r);
+        aq[ks][h + 2 * p] = pack_h2(r[0], r[1]);
+        aq[ks + 2][h + 2 * p] = pack_h2(r[2], r[3]);
       }
   }
+  if (over) atomicOr(a.err, kErrRange);
 }
 
 // B fragments of one n tile of Q . K^T: the 8 ring rows row0 .. row0 + 7,
@@ -104,10 +111,12 @@ __device__ __forceinline__ void qk_mma(const uint32_t (&aq)[4][4], const uint32_
   mma_f16(c, aq[3], b[1][2], b[1][3]);
 }
 
-// acc[0..7] (8 n tiles = 64 dims) += A(16 x 16 key rows) . V rows kb .. kb + 15;
-// all eight B fragments are loaded before the (independent) mma.
+// acc[0..7] (8 n tiles = 64 dims) += (A + Alo)(16 x 16 key rows) . V rows
+// kb .. kb + 15 (the weights as the bf16 pair split_bf16x2 makes); all eight B
+// fragments are loaded before the (independent) mma.
 __device__ __forceinline__ void pv_k16(uint32_t ring_u32, int RB, int kb, int lane,
-                                       const uint32_t (&A)[4], float (&acc)[8][4]) {
+                                       const uint32_t (&A)[4], const uint32_t (&Alo)[4],
+                                       float (&acc)[8][4]) {
   const int slot = (kb + (lane & 15)) & (RB - 1);
   const uint32_t base = ring_u32 + (uint32_t)slot * 128u;
   const int x = slot & 7, m = lane >> 4;
@@ -118,6 +127,8 @@ __device__ __forceinline__ void pv_k16(uint32_t ring_u32, int RB, int kb, int la
   for (int np = 0; np < 4; ++np) {
     mma_bf16(acc[2 * np], A, b[np][0], b[np][1]);
     mma_bf16(acc[2 * np + 1], A, b[np][2], b[np][3]);
+    mma_bf16(acc[2 * np], Alo, b[np][0], b[np][1]);
+    mma_bf16(acc[2 * np + 1], Alo, b[np][2], b[np][3]);
   }
 }
 
@@ -166,7 +177,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
     }
     return;
   }
-  Stager stg{&bar, 0u, a.err};
+  Stager stg = make_stager(&bar, a.err, a.wait_limit, a.stall);
 
   uint32_t aq[2][4][4];
 #pragma unroll
@@ -377,7 +388,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
     const int n_k = (qb + 16 - kr0) >> 4;
     for (int ks = 0; ks < n_k; ++ks) {
       const int kb = kr0 + 16 * ks;
-      uint32_t A[4];
+      uint32_t A[4], Al[4];
 #pragma unroll
       for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -386,21 +397,22 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
           const int lag0 = qb + g + 8 * h - (kb + 2 * tq + 8 * p);   // lag of the first column
           const float v0 = (lag0 >= 0 && lag0 < W) ? er[lag0] : 0.f;
           const float v1 = (lag0 - 1 >= 0 && lag0 - 1 < W) ? er[lag0 - 1] : 0.f;
-          A[h + 2 * p] = pack_bf16x2(v0, v1);
+          split_bf16x2(v0, v1, A[h + 2 * p], Al[h + 2 * p]);
         }
-      pv_k16(ring_u32, RB, kb, lane, A, acc[mt]);
+      pv_k16(ring_u32, RB, kb, lane, A, Al, acc[mt]);
     }
     if (S > 0) {
-      uint32_t A[4];
+      uint32_t A[4], Al[4];
 #pragma unroll
       for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
           const float* er = h ? e_hi : e_lo;
           const int s0 = 2 * tq + 8 * p;
-          A[h + 2 * p] = pack_bf16x2(s0 < S ? er[W + s0] : 0.f, s0 + 1 < S ? er[W + s0 + 1] : 0.f);
+          split_bf16x2(s0 < S ? er[W + s0] : 0.f, s0 + 1 < S ? er[W + s0 + 1] : 0.f, A[h + 2 * p],
+                       Al[h + 2 * p]);
         }
-      pv_k16(sink_u32, 16, 0, lane, A, acc[mt]);
+      pv_k16(sink_u32, 16, 0, lane, A, Al, acc[mt]);
     }
   }
   {
@@ -433,22 +445,28 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
           const float kd = two ? og.w : 1.f, ksu = two ? og.wa : 0.f;
           const float dl = p_lo * kd, sl = p_lo * ksu, dh = p_hi * kd, sh = p_hi * ksu;
           const int kb = qb - og.lo - (two ? 1 : 0);
-          uint32_t A[4];
-          A[0] = pack_bf16x2(bd_lo_c1 ? dl : (bd_c3 ? sl : 0.f), bd_lo_c1 ? sl : (bd_c2 ? dl : 0.f));
-          A[1] = 0u;
-          A[2] = bd_a2 ? pack_bf16x2(sl, 0.f) : 0u;
-          A[3] = pack_bf16x2(bd_lo_c1 ? dh : (bd_c3 ? sh : 0.f), bd_lo_c1 ? sh : (bd_c2 ? dh : 0.f));
-          pv_k16(ring_u32, RB, kb, lane, A, acc[mt]);
+          uint32_t A[4], Al[4];
+          split_bf16x2(bd_lo_c1 ? dl : (bd_c3 ? sl : 0.f), bd_lo_c1 ? sl : (bd_c2 ? dl : 0.f), A[0],
+                       Al[0]);
+          A[1] = Al[1] = 0u;
+          split_bf16x2(bd_a2 ? sl : 0.f, 0.f, A[2], Al[2]);
+          split_bf16x2(bd_lo_c1 ? dh : (bd_c3 ? sh : 0.f), bd_lo_c1 ? sh : (bd_c2 ? dh : 0.f), A[3],
+                       Al[3]);
+          pv_k16(ring_u32, RB, kb, lane, A, Al, acc[mt]);
           if (two) {
             // the 17th row (row a of query 15) as an 8-row k step
-            const uint32_t a1 = bd_a2 ? pack_bf16x2(sh, 0.f) : 0u;
+            uint32_t a1, a1l;
+            split_bf16x2(bd_a2 ? sh : 0.f, 0.f, a1, a1l);
             const int row = kb + 16 + (lane & 7);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
               uint32_t b[4];
               ldsm_x4_t(ring_u32 + swz_off(row, RB, 4 * hh + (lane >> 3)), b);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) mma_bf16_k8(acc[mt][4 * hh + i], 0u, a1, b[i]);
+              for (int i = 0; i < 4; ++i) {
+                mma_bf16_k8(acc[mt][4 * hh + i], 0u, a1, b[i]);
+                mma_bf16_k8(acc[mt][4 * hh + i], 0u, a1l, b[i]);
+              }
             }
           }
         }
@@ -476,7 +494,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
   }
 }
 
-__device__ unsigned g_fwd_tc_err;   // bit 0: a staging wait gave up
+__device__ unsigned g_fwd_tc_err;   // error bits as listed in sa_stage.cuh
 
 int tc_ring_rows(const Problem& pb) {
   int rr = 32;
@@ -533,6 +551,9 @@ cudaError_t launch_fwd_tc(const Problem& pb, const FwdPtrs& p, void* keys_ws, cu
   a.alpha = p.alpha; a.beta = p.beta; a.rope = p.rope;
   a.o = reinterpret_cast<__nv_bfloat16*>(p.o); a.lse = p.lse;
   cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&a.err), g_fwd_tc_err);
+  const WaitCfg wc = wait_cfg();
+  a.wait_limit = wc.limit;
+  a.stall = wc.stall;
   if (e != cudaSuccess) return e;
   if ((e = make_rows_map(&a.tmK, keys_ws, pb.T, pb.units())) != cudaSuccess) return e;
   if ((e = make_rows_map(&a.tmV, p.v, pb.T, pb.units())) != cudaSuccess) return e;

@@ -51,6 +51,15 @@ sa_status validate_params(const sa_params* p, Problem* pb);
 cudaError_t launch_fwd_dispatch(const Problem& pb, const FwdPtrs& a, cudaStream_t st,
                                 int* launches);
 
+// Diagnostics of the bounded staging waits (sa_api.cu): the wait limit in SM
+// clocks (0: the kernels' default) and whether launches plant a stall in
+// their first staging round (sparse_attn_set_wait_limit / _plant_stall).
+struct WaitCfg {
+  long long limit;
+  int stall;
+};
+WaitCfg wait_cfg();
+
 // Tracing hook: brackets one kernel launch with events when tracing is on.
 // Call with begin = true just before the launch and false just after it.
 void trace_mark(const char* kernel, cudaStream_t st, bool begin);
@@ -91,6 +100,8 @@ cudaError_t fast_bwd_read_error(unsigned* out, bool clear);
 // [units][T][64] array, row r rotated at position r % T.
 cudaError_t launch_rope_rows(const void* x, const float2* rope, int T, long long n_rows, float mul,
                              void* y, cudaStream_t st, const char* trace_name);
+// The pre-pass's error word (bit 2: a finite rotated value beyond fp16's range).
+cudaError_t prep_read_error(unsigned* out, bool clear);
 
 // Staged bf16 / D=64 backward (sa_fast_bwd.cu).
 bool fast_bwd_supported(const Problem& pb);

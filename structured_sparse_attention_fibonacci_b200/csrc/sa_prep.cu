@@ -15,11 +15,12 @@ namespace {
 using namespace fast;
 
 // One thread per (row, RoPE pair-chunk p): dims [8p, 8p+8) pair with
-// [32+8p, 32+8p+8).
+// [32+8p, 32+8p+8).  A finite rotated value that overflows fp16 sets bit 2
+// of the error word (the staged kernels' range limit).
 __global__ void __launch_bounds__(256) k_rope_rows(const __nv_bfloat16* __restrict__ X,
                                                    const float2* __restrict__ rope, int T,
                                                    long long n_rows, float mul,
-                                                   __half* __restrict__ Y) {
+                                                   __half* __restrict__ Y, unsigned* err) {
   const long long task = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (task >= n_rows * 4) return;
   const long long row = task >> 2;
@@ -39,10 +40,13 @@ __global__ void __launch_bounds__(256) k_rope_rows(const __nv_bfloat16* __restri
     x1[h + 1] = (a1 * t.z - b1 * t.w) * mul;
     x2[h + 1] = (b1 * t.z + a1 * t.w) * mul;
   }
+  if (half_overflow8(x1) | half_overflow8(x2)) atomicOr(err, 4u);
   uint4* y = reinterpret_cast<uint4*>(Y + row * kD);
   y[p] = pack8_h(x1);
   y[p + 4] = pack8_h(x2);
 }
+
+__device__ unsigned g_prep_err;   // bit 2: a rotated value beyond fp16's range
 
 }  // namespace
 
@@ -51,11 +55,21 @@ cudaError_t launch_rope_rows(const void* x, const float2* rope, int T, long long
   if (n_rows <= 0) return cudaSuccess;
   const long long tasks = n_rows * 4;
   const unsigned grid = (unsigned)((tasks + 255) / 256);
+  unsigned* err = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_prep_err);
+  if (e != cudaSuccess) return e;
   trace_mark(trace_name, st, true);
   k_rope_rows<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x), rope, T, n_rows,
-                                    mul, reinterpret_cast<__half*>(y));
+                                    mul, reinterpret_cast<__half*>(y), err);
   trace_mark(trace_name, st, false);
   return cudaGetLastError();
+}
+
+cudaError_t prep_read_error(unsigned* out, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_prep_err, sizeof(unsigned));
+  if (e != cudaSuccess || !clear || *out == 0) return e;
+  const unsigned zero = 0;
+  return cudaMemcpyToSymbol(g_prep_err, &zero, sizeof(unsigned));
 }
 
 }  // namespace sa

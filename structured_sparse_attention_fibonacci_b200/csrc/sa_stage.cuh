@@ -17,6 +17,14 @@
 //
 // Rows outside [0, T) are zero-filled by the threads (the first and last tile
 // of a sequence), so every slot a lane reads holds finite data.
+//
+// Device error word bits (shared by every staged kernel):
+//   bit 0 (kErrWait)   a bounded wait for a staging round gave up;
+//   bit 1 (kErrBounds) a row index outside the rows staged, or a staging round
+//                      larger than the ring (checked only in builds with
+//                      SA_DEBUG_BOUNDS; the access is then skipped or clamped);
+//   bit 2 (kErrRange)  a finite input whose 16-bit staged form overflows
+//                      (|RoPE(K)| / 256 or a scaled query beyond fp16's 65504).
 #pragma once
 
 #include "sa_fast_common.cuh"
@@ -29,9 +37,11 @@ using fast::kD;
 
 constexpr int kMirror = 12;          // mirrored slots after the ring (longest run: 11 rows)
 constexpr int kRowBytes = 128;       // 64 x 16-bit
-// Bounded waits: a wait that has not completed after this many SM clocks
-// (about half a second) gives up and reports through the device error word.
+// Bounded waits: by default a wait that has not completed after this many SM
+// clocks (about half a second) gives up and reports through the device error
+// word; the host can lower the limit (sparse_attn_set_wait_limit).
 constexpr long long kWaitClocks = 1000000000LL;
+constexpr unsigned kErrWait = 1u, kErrBounds = 2u, kErrRange = 4u;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -90,12 +100,66 @@ __device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t b
 }
 
 // Staging state of one CTA: the barrier and its phase bit (identical in every
-// thread) and the device error word.
+// thread), the device error word, the wait limit in SM clocks and the planted
+// stall of the failure-path test (sparse_attn_plant_stall: the first round
+// expects 16 bytes that no copy delivers, so its wait must give up).  In
+// SA_DEBUG_BOUNDS builds it also tracks the rows [vlo, vhi) the ring holds.
 struct Stager {
   uint64_t* bar;
   uint32_t phase;
   unsigned* err;
+  long long limit;
+  int stall;
+#ifdef SA_DEBUG_BOUNDS
+  int vlo, vhi;
+#endif
 };
+
+__device__ __forceinline__ Stager make_stager(uint64_t* bar, unsigned* err, long long limit,
+                                              int stall) {
+  Stager s;
+  s.bar = bar;
+  s.phase = 0u;
+  s.err = err;
+  s.limit = limit > 0 ? limit : kWaitClocks;
+  s.stall = stall;
+#ifdef SA_DEBUG_BOUNDS
+  s.vlo = s.vhi = 0;
+#endif
+  return s;
+}
+
+// SA_DEBUG_BOUNDS: record a bounds error (bit 1) when rows [r0, r1) are not
+// all among the rows the ring holds; other builds: nothing.
+__device__ __forceinline__ void dbg_rows(const Stager& s, int r0, int r1) {
+#ifdef SA_DEBUG_BOUNDS
+  if (r0 < s.vlo || r1 > s.vhi) atomicOr(s.err, kErrBounds);
+#else
+  (void)s; (void)r0; (void)r1;
+#endif
+}
+
+// SA_DEBUG_BOUNDS: record a bounds error when cond is false.
+__device__ __forceinline__ void dbg_check(unsigned* err, bool cond) {
+#ifdef SA_DEBUG_BOUNDS
+  if (!cond) atomicOr(err, kErrBounds);
+#else
+  (void)err; (void)cond;
+#endif
+}
+
+// SA_DEBUG_BOUNDS: the ring now also holds rows [a, b): extend the tracked
+// range when the round is adjacent to it (rows below, or above, what it
+// held), keeping the RB rows nearest the new ones; else restart from [a, b).
+__device__ __forceinline__ void dbg_staged(Stager& s, int RB, int a, int b) {
+#ifdef SA_DEBUG_BOUNDS
+  if (b == s.vlo && s.vlo < s.vhi) { s.vlo = a; s.vhi = min(s.vhi, a + RB); }
+  else if (a == s.vhi && s.vlo < s.vhi) { s.vhi = b; s.vlo = max(s.vlo, b - RB); }
+  else { s.vlo = a; s.vhi = b; }
+#else
+  (void)s; (void)RB; (void)a; (void)b;
+#endif
+}
 
 // One staging round: any number of stage_ring / stage_plain calls (thread 0
 // registers their bytes and issues their copies; every thread zero-fills),
@@ -103,19 +167,23 @@ struct Stager {
 // is registered, so the phase cannot complete early; a round without copies
 // completes at the arrival.
 
-// Arrive (thread 0) and wait for the round, at most kWaitClocks; ends with a
+// Arrive (thread 0) and wait for the round, at most s.limit clocks; ends with a
 // CTA barrier, so the zero-fills are visible too.  Returns nonzero in every
 // thread when any thread gave up (the error word gets bit 0); the caller then
 // calls stage_drain and returns.
 __device__ __forceinline__ int stage_commit_wait(Stager& s) {
-  if (threadIdx.x == 0) mbar_arrive(s.bar);
+  if (threadIdx.x == 0) {
+    if (s.stall) mbar_expect_tx(s.bar, 16u);   // planted: bytes no copy delivers
+    mbar_arrive(s.bar);
+  }
+  s.stall = 0;
   const long long t0 = clock64();
   bool ok;
   while (!(ok = mbar_try_wait(s.bar, s.phase)))
-    if (clock64() - t0 > kWaitClocks) break;
+    if (clock64() - t0 > s.limit) break;
   s.phase ^= 1u;
   const int bad = __syncthreads_or(!ok);
-  if (bad && threadIdx.x == 0) atomicOr(s.err, 1u);
+  if (bad && threadIdx.x == 0) atomicOr(s.err, kErrWait);
   return bad;
 }
 
@@ -124,7 +192,7 @@ __device__ __forceinline__ int stage_commit_wait(Stager& s) {
 __device__ __forceinline__ void stage_drain(Stager& s) {
   const long long t0 = clock64();
   while (!mbar_try_wait(s.bar, s.phase ^ 1u))
-    if (clock64() - t0 > kWaitClocks) break;
+    if (clock64() - t0 > s.limit) break;
 }
 
 // Stage rows [a, b) (b - a <= RB) of `src` (a 16-bit [T][64] array) into the
@@ -133,6 +201,13 @@ __device__ __forceinline__ void stage_drain(Stager& s) {
 // last reads of the slots involved.
 __device__ __forceinline__ void stage_ring(Stager& s, unsigned char* ring, int RB, const void* src,
                                            int T, int a, int b) {
+#ifdef SA_DEBUG_BOUNDS
+  if (b - a > RB) {                   // more rows than slots: record and stage none
+    if (threadIdx.x == 0) atomicOr(s.err, kErrBounds);
+    return;
+  }
+#endif
+  dbg_staged(s, RB, a, b);
   const int ca = max(a, 0), cb = min(b, T);
   {
     const int n_lo = max(0, min(b, 0) - a);          // rows a .. min(b, 0) - 1

@@ -83,6 +83,19 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// Two fp32 values as a bf16 pair rounded to nearest (hi) plus the bf16 pair of
+// what that rounding left (lo): hi + lo holds each value to about 2^-17 of
+// itself, where hi alone is off by up to 2^-9.  The P.V products run on
+// bf16 tensor cores (V is bf16); feeding them both halves of the weights keeps
+// the output's error at fp32-accumulation level.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
 // Byte offset, within the ring, of 16-byte chunk `ch` of row `row`.
 __device__ __forceinline__ uint32_t swz_off(int row, int RB, int ch) {
   const int slot = row & (RB - 1);
@@ -106,6 +119,13 @@ __device__ __forceinline__ void tma_rows8(uint32_t dst, const CUtensorMap* map, 
 // barrier (stage::stage_commit_wait).
 __device__ __forceinline__ void stage_tiles(Stager& s, uint32_t ring_u32, int RB,
                                             const CUtensorMap* map, int unit, int a, int b) {
+#ifdef SA_DEBUG_BOUNDS
+  if (b - a > RB || (a & 7) || (b & 7)) {   // beyond the ring, or not whole boxes: stage none
+    if (threadIdx.x == 0) atomicOr(s.err, stage::kErrBounds);
+    return;
+  }
+#endif
+  stage::dbg_staged(s, RB, a, b);
   if (threadIdx.x != 0 || a >= b) return;
   stage::mbar_expect_tx(s.bar, (uint32_t)(b - a) * 128u);
   for (int r = a; r < b; r += 8)

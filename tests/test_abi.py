@@ -39,13 +39,18 @@ def test_header_declares_the_boundary():
             "sparse_attn_status_string"} <= names
 
 
-def test_every_declared_symbol_is_exported(lib):
-    out = subprocess.check_output(["nm", "-D", "--defined-only", sa.LIB_PATH]).decode()
+@pytest.mark.parametrize("path", [sa.LIB_PATH, sa.BOUNDS_LIB_PATH], ids=["library", "bounds"])
+def test_every_declared_symbol_is_exported(lib, path):
+    """Both builds (the library and its bounds-checking variant) export every
+    function the header declares."""
+    out = subprocess.check_output(["nm", "-D", "--defined-only", path]).decode()
     exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
     missing = declared_functions() - exported
     assert not missing, missing
+    other = ctypes.CDLL(path)
     for name in declared_functions():
         assert getattr(lib, name) is not None
+        assert getattr(other, name) is not None
 
 
 def test_binding_lists_every_export():

@@ -8,19 +8,41 @@ from structured_sparse_attention_fibonacci_b200.inputs import WORKLOADS
 
 
 def test_algorithmic_bytes_per_token_head():
-    # forward: Q, K, V read and O written (4 rows of 64 bf16), LSE 4 B
-    assert bench.alg_bytes_per_token_head("fwd_fast", 64, 2) == 4 * 128 + 4
-    assert bench.alg_bytes_per_token_head("fwd_tc", 64, 2) == 516
-    # the saving forward also writes its context; the prior adds its 4 B
-    assert bench.alg_bytes_per_token_head("fwd_fast", 64, 2, context=296) == 812
-    assert bench.alg_bytes_per_token_head("fwd_fast", 64, 2, prior=True) == 520
-    # query and key sides: six rows and two fp32 values each
-    assert bench.alg_bytes_per_token_head("bwd_q_fast", 64, 2) == 6 * 128 + 8
-    assert bench.alg_bytes_per_token_head("bwd_q_fast", 64, 2, prior=True) == 784
-    assert bench.alg_bytes_per_token_head("bwd_kv_fast", 64, 2) == 776
-    # the RoPE pre-pass reads a row and writes it rotated; reductions count 0
-    assert bench.alg_bytes_per_token_head("rope_keys", 64, 2) == 256
+    """The roofline bytes follow the problem's definition: the forward's unique
+    Q, K, V and O (512 B per token-head at d = 64, bf16) and the backward's
+    Q, K, V, O, dO, dQ, dK, dV and LSE (1028 B), split between the two
+    backward kernels as they touch the tensors; intermediates count 0."""
+    assert bench.alg_bytes_per_token_head("fwd_fast", 64, 2) == 4 * 128 == 512
+    assert bench.alg_bytes_per_token_head("fwd_tc", 64, 2) == 512
+    assert bench.alg_bytes_per_token_head("fwd_fast", 64, 2, prior=True) == 516
+    # query side: Q, K, V, dO, LSE read, dQ written; key side: dK, dV written, O
+    assert bench.alg_bytes_per_token_head("bwd_q_fast", 64, 2) == 5 * 128 + 4 == 644
+    assert bench.alg_bytes_per_token_head("bwd_kv_fast", 64, 2) == 3 * 128 == 384
+    assert (bench.alg_bytes_per_token_head("bwd_q_fast", 64, 2)
+            + bench.alg_bytes_per_token_head("bwd_kv_fast", 64, 2)
+            == bench.phase_bytes_per_token_head("backward", 64, 2) == 1028)
+    assert bench.phase_bytes_per_token_head("forward", 64, 2) == 512
+    assert bench.phase_bytes_per_token_head("forward", 16, 4) == 256      # the fp32 d = 16 case
+    # pre-passes, the training context and reductions are intermediates
+    assert bench.alg_bytes_per_token_head("rope_keys", 64, 2) == 0
     assert bench.alg_bytes_per_token_head("reduce_dalpha", 64, 2) == 0
+
+
+def test_distinct_rows_and_flops():
+    """At alpha = 1 the Fibonacci ladder's lags 1, 2, 3, 5, 8 fall in the
+    window of 12 and 13 .. 987 add 10 rows (integer distances read one row);
+    a non-integer alpha reads both rows of every far offset."""
+    assert bench.distinct_rows(1.0, WORKLOADS["paper_fwd"].offsets, 12, 0) == 22
+    assert bench.distinct_rows(1.0, WORKLOADS["long_sinks"].offsets, 64, 4) == 64 + 6 + 4
+    # alpha = 1.1234: lags 1, 2, 3, 5, 8, 14 lie in or next to the window
+    n = bench.distinct_rows(1.1234, WORKLOADS["paper_fwd"].offsets, 12, 0)
+    assert 12 + 2 * 8 <= n <= 12 + 2 * 10
+    wl = WORKLOADS["tiny_fp32"]
+    assert bench.alg_flops(wl, "forward") == 4 * 16 * bench.distinct_rows(1.0, wl.offsets, 6, 0) * 128
+    lt = WORKLOADS["learned_train"]
+    assert bench.alg_flops(lt, "backward") == 2 * bench.alg_flops(lt, "forward")
+    assert (bench.kernel_flops(lt, "bwd_q_fast") + bench.kernel_flops(lt, "bwd_kv_fast")
+            == bench.alg_flops(lt, "backward"))
 
 
 def test_decode_bytes_count_every_member_row():
