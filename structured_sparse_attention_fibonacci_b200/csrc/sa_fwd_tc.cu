@@ -92,17 +92,6 @@ __device__ __forceinline__ void q_frags(const TcFwdArgs& a, const __nv_bfloat16*
   if (over) atomicOr(a.err, kErrRange);
 }
 
-// B fragments of one n tile of Q . K^T: the 8 ring rows row0 .. row0 + 7,
-// k steps 0..3 as b[kp][0..1] (k step 2 kp) and b[kp][2..3] (k step 2 kp + 1).
-__device__ __forceinline__ void qk_load(uint32_t ring_u32, int RB, int row0, int lane,
-                                        uint32_t (&b)[2][4]) {
-  const int slot = (row0 + (lane & 7)) & (RB - 1);
-  const uint32_t base = ring_u32 + (uint32_t)slot * 128u;
-  const int x = slot & 7, m = lane >> 3;
-  ldsm_x4(base + (uint32_t)((m ^ x) << 4), b[0]);
-  ldsm_x4(base + (uint32_t)(((4 + m) ^ x) << 4), b[1]);
-}
-
 __device__ __forceinline__ void qk_mma(const uint32_t (&aq)[4][4], const uint32_t (&b)[2][4],
                                        float (&c)[4]) {
   mma_f16(c, aq[0], b[0][0], b[0][1]);

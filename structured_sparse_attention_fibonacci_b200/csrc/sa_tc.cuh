@@ -132,6 +132,18 @@ __device__ __forceinline__ void stage_tiles(Stager& s, uint32_t ring_u32, int RB
     tma_rows8(ring_u32 + (uint32_t)((r & (RB - 1)) * 128), map, r, unit, s.bar);
 }
 
+// B fragments of one n tile of A . X^T for 8 swizzled ring rows row0 ..
+// row0 + 7 of a 16-bit [T][64] array: k steps 0..3 (dims 16 ks ..) as
+// b[kp][0..1] (k step 2 kp) and b[kp][2..3] (k step 2 kp + 1).
+__device__ __forceinline__ void qk_load(uint32_t ring_u32, int RB, int row0, int lane,
+                                        uint32_t (&b)[2][4]) {
+  const int slot = (row0 + (lane & 7)) & (RB - 1);
+  const uint32_t base = ring_u32 + (uint32_t)slot * 128u;
+  const int x = slot & 7, m = lane >> 3;
+  ldsm_x4(base + (uint32_t)((m ^ x) << 4), b[0]);
+  ldsm_x4(base + (uint32_t)(((4 + m) ^ x) << 4), b[1]);
+}
+
 __device__ __forceinline__ int floor8(int x) { return x & ~7; }
 __device__ __forceinline__ int ceil8(int x) { return (x + 7) & ~7; }
 __device__ __forceinline__ int floor16(int x) { return x & ~15; }
