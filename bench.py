@@ -54,6 +54,9 @@ FALLBACK_HBM_GBS = 6650.0
 B200_SMS, FP32_LANES_PER_SM = 148, 128
 # Configurations timed beside the headline in the "workloads" record: the
 # other four problem-statement configurations and the power-of-2 control.
+# --forward: which bf16 / head-dim-64 forward kernel the plain forwards run
+# (sparse_attn_select_forward; the training forward is always the CUDA-core one)
+FORWARD_KERNELS = {"auto": 0, "cuda_core": 1, "mma_sync": 2, "tcgen05": 3}
 OTHER_WORKLOADS = ("tiny_fp32", "paper_fwd", "extrap_4x", "long_sinks", "pow2_extrap")
 
 
@@ -481,6 +484,7 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    sa.select_forward(FORWARD_KERNELS[args.forward])
     wl = WORKLOADS[args.workload]
     wl_rank = wl.shrink(seed=wl.seed + 100000 * rank) if world > 1 else wl
     host = make_inputs(wl_rank, pin=True)
@@ -882,6 +886,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the forward timings of the other configurations")
+    ap.add_argument("--forward", choices=tuple(FORWARD_KERNELS), default="auto",
+                    help="forward kernel of the plain (non-training) forwards")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--reference-budget-s", type=float, default=120.0)
     args = ap.parse_args()

@@ -338,11 +338,15 @@ void sparse_attn_force_general(int on);
 /*
  * Diagnostics: which bf16 / D = 64 forward kernel sparse_attn_fwd runs.
  * 0 (default): the faster for the configuration, as measured on B200: the
- * tensor-core kernel for windows of 32 or more, except where its shared
+ * tensor-core kernel for windows of 48 or more, except where its shared
  * memory would leave it one CTA per SM while the CUDA-core kernel keeps two;
  * otherwise the CUDA-core kernel.  1: the CUDA-core staged kernel; 2: the
- * tensor-core kernel where it applies (at most 16 sinks).  Other values mean
- * 0.  Process wide; sparse_attn_force_general takes precedence.
+ * warp-level (mma.sync) tensor-core kernel where it applies (at most 16
+ * sinks); 3: the fifth-generation tensor-core kernel (tcgen05 GEMMs for the
+ * window band and the sinks, accumulators in tensor memory, offset members on
+ * the CUDA cores) where it applies (at most 16 sinks, band plus sinks at most
+ * 256 rows: W <= 113 with sinks, W <= 129 without), else as 0.  Other values
+ * mean 0.  Process wide; sparse_attn_force_general takes precedence.
  */
 void sparse_attn_select_forward(int which);
 

@@ -172,7 +172,8 @@ def force_general(on: bool = True) -> None:
 
 def select_forward(which: int = 0) -> None:
     """Diagnostics: bf16 / d=64 forward kernel choice (0 auto, 1 CUDA-core
-    staged, 2 tensor-core); see sparse_attn_select_forward."""
+    staged, 2 tensor-core mma.sync, 3 tensor-core tcgen05); see
+    sparse_attn_select_forward."""
     lib().sparse_attn_select_forward(int(which))
 
 

@@ -15,7 +15,7 @@ namespace {
 
 thread_local int32_t g_last_launches = 0;
 int g_force_general = 0;  // diagnostics: route every call through the general kernels
-int g_fwd_select = 0;     // diagnostics: 0 auto, 1 CUDA-core staged forward, 2 tensor-core forward
+int g_fwd_select = 0;     // diagnostics: 0 auto, 1 CUDA-core staged, 2 mma.sync, 3 tcgen05 forward
 long long g_wait_limit = 0;  // diagnostics: staging wait limit in SM clocks (0: default)
 int g_plant_stall = 0;       // diagnostics: failure-path test of the bounded waits
 
@@ -153,7 +153,9 @@ int32_t sparse_attn_last_launch_count(void) { return g_last_launches; }
 
 void sparse_attn_force_general(int on) { g_force_general = on != 0; }
 
-void sparse_attn_select_forward(int which) { g_fwd_select = (which == 1 || which == 2) ? which : 0; }
+void sparse_attn_select_forward(int which) {
+  g_fwd_select = (which >= 1 && which <= 3) ? which : 0;
+}
 
 void sparse_attn_set_wait_limit(long long clocks) { g_wait_limit = clocks > 0 ? clocks : 0; }
 
@@ -192,13 +194,14 @@ int32_t sparse_attn_trace_read(int32_t max, const char** names, double* total_ms
 }
 
 int32_t sparse_attn_device_error(int clear) {
-  unsigned fwd = 0, fwd_tc = 0, bwd = 0, prep = 0;
+  unsigned fwd = 0, fwd_tc = 0, fwd_umma = 0, bwd = 0, prep = 0;
   if (sa::fast_fwd_read_error(&fwd, clear != 0) != cudaSuccess ||
       sa::fast_fwd_tc_read_error(&fwd_tc, clear != 0) != cudaSuccess ||
+      sa::fwd_umma_read_error(&fwd_umma, clear != 0) != cudaSuccess ||
       sa::fast_bwd_read_error(&bwd, clear != 0) != cudaSuccess ||
       sa::prep_read_error(&prep, clear != 0) != cudaSuccess)
     return -1;
-  return (int32_t)(fwd | fwd_tc | bwd | prep);
+  return (int32_t)(fwd | fwd_tc | fwd_umma | bwd | prep);
 }
 
 size_t sparse_attn_workspace_size(const sa_params* p, int backward) {
@@ -237,6 +240,8 @@ sa_status fwd_impl(const sa_params* p, const void* q, const void* k, const void*
   cudaError_t e;
   if (g_force_general || !sa::fast_fwd_supported(pb))
     e = sa::launch_fwd_general(pb, a, st, &launches);
+  else if (g_fwd_select == 3 && sa::umma_fwd_supported(pb))
+    e = sa::launch_fwd_umma(pb, a, workspace, st, &launches);
   else if (g_fwd_select == 2 ? sa::tc_fwd_supported(pb)
                               : (g_fwd_select == 0 && sa::tc_fwd_preferred(pb)))
     e = sa::launch_fwd_tc(pb, a, workspace, st, &launches);

@@ -515,12 +515,12 @@ static int ctas_per_sm(size_t smem) {
   return (int)std::min<size_t>(4, (size_t)(228 * 1024) / per);
 }
 
-// Measured on B200 (B=1 H=16 T=32768 with 4 sinks, and B=2 H=8 T=4096):
-// - the tensor-core forward is faster from W = 32 up (by 18-38% at W = 64..112);
-// - it is slower where its larger ring leaves it one CTA per SM and the
-//   CUDA-core forward keeps two (W = 128: 0.95 vs 0.87 ms).
+// Measured on B200 (B=1 H=16 T=32768 d=64, 4 sinks, alpha = 1 and 1.1234,
+// windows 16..128): the CUDA-core forward is faster up to W = 40 (by 4-17%),
+// this one from W = 48 (by 2-4% at 48..56, 8-27% at 64..112); at W = 128 its
+// ring leaves it one CTA per SM and it is the slower (1.02 vs 0.83 ms).
 bool tc_fwd_preferred(const Problem& pb) {
-  if (!tc_fwd_supported(pb) || pb.W < 32) return false;
+  if (!tc_fwd_supported(pb) || pb.W < 48) return false;
   const int tc = ctas_per_sm(tc_fwd_smem(pb, nullptr, nullptr));
   const int cc = fast_fwd_supported(pb) ? ctas_per_sm(fast_fwd_smem(pb, nullptr, nullptr)) : 0;
   return !(tc == 1 && cc >= 2);

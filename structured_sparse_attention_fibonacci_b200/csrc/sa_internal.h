@@ -82,14 +82,25 @@ cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& a, void* keys_ws, 
 // Tensor-core bf16 / D=64 forward (sa_fwd_tc.cu); keys_ws as for the staged
 // forward (fast_fwd_workspace bytes, required).
 bool tc_fwd_supported(const Problem& pb);
-// Where the tensor-core forward is the faster one: windows of 32 and more,
+// Where the tensor-core forward is the faster one: windows of 48 and more,
 // except where its shared memory leaves it one CTA per SM while the CUDA-core
-// forward keeps two (measured on B200; W = 12 is 9% slower on tensor cores).
+// forward keeps two (measured on B200; at W = 12 it runs 25% slower).
 bool tc_fwd_preferred(const Problem& pb);
 size_t tc_fwd_smem(const Problem& pb, int* ring_rows, int* sc_stride);
 cudaError_t launch_fwd_tc(const Problem& pb, const FwdPtrs& a, void* keys_ws, cudaStream_t st,
                           int* launches);
 cudaError_t fast_fwd_tc_read_error(unsigned* out, bool clear);
+// Fifth-generation tensor-core bf16 / D=64 forward (sa_fwd_umma.cu): the
+// window band and the sinks as tcgen05 GEMMs with accumulators in tensor
+// memory, the offset members on the CUDA cores; keys_ws as for the staged
+// forward.  Applies while the band plus 16 sink rows is at most 256 rows
+// (W <= 113 with sinks, 129 without) and S <= 16.  Runs only when selected
+// (sparse_attn_select_forward(3)): measured on B200 it is within 4% of the
+// mma.sync forward at W = 64..112 and slower elsewhere.
+bool umma_fwd_supported(const Problem& pb);
+cudaError_t launch_fwd_umma(const Problem& pb, const FwdPtrs& a, void* keys_ws, cudaStream_t st,
+                            int* launches);
+cudaError_t fwd_umma_read_error(unsigned* out, bool clear);
 
 // Device error words of the staged kernels (bit 0: a bounded staging wait
 // gave up); optionally cleared after reading.

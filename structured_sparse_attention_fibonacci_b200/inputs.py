@@ -100,6 +100,14 @@ WORKLOADS = {
                                  "W=12"),
     "long_sinks": Workload("long_sinks", 1, 1, 16, 32768, 64, 64, 4, torch.bfloat16, "fixed", 5000,
                            note="B=1 H=16 T=32768 d=64 bf16, W=64, 4 sinks, alpha=1"),
+    # forward-kernel comparisons across window lengths (the CUDA-core, mma.sync
+    # and tcgen05 forwards); not among the five benchmark configurations
+    "window_32": Workload("window_32", 1, 1, 16, 32768, 64, 32, 4, torch.bfloat16, "fixed", 5100,
+                          note="B=1 H=16 T=32768 d=64 bf16, W=32, 4 sinks, alpha=1"),
+    "window_64_stagger": Workload("window_64_stagger", 4, 1, 4, 32768, 64, 64, 4, torch.bfloat16,
+                                  "linear", 5200,
+                                  note="4 layers B=1 H=4 T=32768 d=64 bf16, W=64, 4 sinks, "
+                                       "linear stagger (interpolated offsets)"),
     "pi_skip": Workload("pi_skip", 16, 8, 8, 1024, 64, 5, 0, torch.bfloat16, "fixed", 7000,
                         offsets=(16,),
                         note="periodic skip in autoregressive form: local window of the "

@@ -45,7 +45,7 @@ def stalled():
         sa.device_error(clear=True)
 
 
-@pytest.mark.parametrize("kernel", [1, 2], ids=["cuda_core", "tensor_core"])
+@pytest.mark.parametrize("kernel", [1, 2, 3], ids=["cuda_core", "tensor_core", "tcgen05"])
 def test_forward_wait_gives_up_and_reports(stalled, kernel):
     q, k, v, _ = _inputs((1, 1, 2, 300, 64), seed=21)
     alpha = torch.tensor([1.1234], device=DEV)

@@ -157,6 +157,31 @@ def test_full_workload_sampled(name, mode):
     check_dalpha(grads[3], ref[3], wl.dtype, f"{name} {mode} dalpha", units=ref.units)
 
 
+@pytest.mark.parametrize("name", ["long_sinks", "window_64_stagger", "paper_fwd"])
+def test_tcgen05_forward_full_size(name):
+    """The fifth-generation tensor-core forward (selected explicitly; the
+    default dispatch does not take it) at full size, sampled units."""
+    wl = WORKLOADS[name]
+    q, k, v = make_inputs(wl, device=DEV)[:3]
+    alpha = wl.alpha().to(DEV)
+    kw = dict(window=wl.window, sinks=wl.sinks, offsets=wl.offsets, rope_base=wl.rope_base)
+    sa.select_forward(3)
+    sa.trace_enable(True)
+    try:
+        o, lse = sa.fwd(q, k, v, alpha, **kw)
+        torch.cuda.synchronize()
+        names = set(sa.trace_read())
+    finally:
+        sa.trace_enable(False)
+        sa.select_forward(0)
+    assert "fwd_umma" in names, names
+    assert sa.device_error() == 0
+    for (l, b, h) in _sample_units(wl, 4):
+        sl = (slice(l, l + 1), slice(b, b + 1), slice(h, h + 1))
+        o_ref, lse_ref = oracle_fwd(q[sl], k[sl], v[sl], alpha[l:l + 1], **kw)
+        check_fwd(o[sl], lse[sl], o_ref, lse_ref, wl.dtype, f"{name} tcgen05 unit {(l, b, h)}")
+
+
 # ---- the staged bf16 d=64 forward and the general kernels on the same inputs ----
 FAST = [
     ("fast_tail_129", (2, 1, 2, 129, 64), 12, 0, [0.5, 1.5], FIB15),
@@ -176,7 +201,7 @@ FAST = [
 ]
 
 
-@pytest.mark.parametrize("kernel", [1, 2], ids=["cuda_core", "tensor_core"])
+@pytest.mark.parametrize("kernel", [1, 2, 3], ids=["cuda_core", "tensor_core", "tcgen05"])
 @pytest.mark.parametrize("case", FAST, ids=[c[0] for c in FAST])
 def test_fast_and_general_forward(case, kernel):
     name, shape, W, S, alphas, offs = case
@@ -225,6 +250,15 @@ def test_fast_path_is_the_one_dispatched():
         sa.trace_enable(False)
         sa.select_forward(0)
     assert names == {"rope_keys", "fwd_tc"}, names
+    sa.select_forward(3)
+    sa.trace_enable(True)
+    try:
+        run_gpu_fwd(q, k, v, alpha, window=12)
+        names = set(sa.trace_read())
+    finally:
+        sa.trace_enable(False)
+        sa.select_forward(0)
+    assert names == {"rope_keys", "fwd_umma"}, names
 
 
 @pytest.mark.parametrize("case", FAST, ids=[c[0] for c in FAST])
@@ -352,7 +386,7 @@ def _scaled_inputs(shape, c, seed):
     return [t.to(torch.bfloat16).to(DEV) for t in (q * c, k * c, v, do)]
 
 
-@pytest.mark.parametrize("kernel", [1, 2], ids=["cuda_core", "tensor_core"])
+@pytest.mark.parametrize("kernel", [1, 2, 3], ids=["cuda_core", "tensor_core", "tcgen05"])
 def test_staged_path_at_twice_the_input_scale(kernel):
     shape = (2, 1, 2, 600, 64)
     q, k, v, do = _scaled_inputs(shape, 2.0, seed=505)

@@ -134,7 +134,7 @@ def test_prior_general_kernels_forced():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("kernel", [1, 2])
+@pytest.mark.parametrize("kernel", [1, 2, 3])
 def test_prior_on_both_staged_forwards(kernel):
     """W = 64 with sinks: the tensor-core forward (the default there) and the
     CUDA-core forward both carry the prior; each is dispatched as selected and
@@ -152,7 +152,7 @@ def test_prior_on_both_staged_forwards(kernel):
         sa.trace_enable(False)
     finally:
         sa.select_forward(0)
-    assert ("fwd_tc" if kernel == 2 else "fwd_fast") in names, names
+    assert {1: "fwd_fast", 2: "fwd_tc", 3: "fwd_umma"}[kernel] in names, names
     o_ref, lse_ref = oracle_fwd(q, k, v, alpha, beta=to_np(beta), **kw)
     check_fwd(o, lse, o_ref, lse_ref, torch.bfloat16, f"prior forward kernel {kernel}")
 
