@@ -220,7 +220,7 @@ def time_forward_workload(sa, torch, dev, name, steps, warmup, peak, alu_peak):
            if small else "inputs larger than L2",
            "kernels_ms": kern, "alg_bytes_per_token_head": bpt,
            "hbm": {"achieved_GBps": gbs, "frac": gbs / peak, "kernel": fwd_k,
-                   "kernel_frac": k_gbs / peak},
+                   "kernel_frac": k_gbs / peak, **workload_traffic(wl.name, fwd_k)},
            "alu": {"alg_flops": fl, "achieved_TFLOPs": fl / (ms / 1e3) / 1e12,
                    "frac": fl / (ms / 1e3) / 1e12 / alu_peak if alu_peak else None}}
     del q, k, v, o, lse, ws, flush
@@ -241,14 +241,24 @@ def decode_bytes_per_token_head(wl, elt):
 # capture per entry; keyed by workload, kernel and the hash of the kernel
 # sources the capture ran (kernel_source_hash): a changed source reports null.
 MEASURED_TRAFFIC = {
-    "learned_train/bwd_q_fast@6a730910219c": 779.8,
-    "pi_gate_train/bwd_q_fast@6a730910219c": 545.4,
-    "paper_fwd/fwd_fast@6a730910219c": 494.5,
-    "extrap_4x/fwd_fast@6a730910219c": 496.4,
-    "pi_skip/fwd_fast@6a730910219c": 492.7,
-    "long_sinks/fwd_tc@6a730910219c": 509.0,
-    "decode_4k/decode@6a730910219c": 8121.8,
+    "learned_train/bwd_q_fast@096d815d8754": 780.6,
+    "pi_gate_train/bwd_q_fast@096d815d8754": 545.5,
+    "paper_fwd/fwd_fast@096d815d8754": 494.2,
+    "extrap_4x/fwd_fast@096d815d8754": 495.8,
+    "pow2_extrap/fwd_fast@096d815d8754": 496.6,
+    "pi_skip/fwd_fast@096d815d8754": 491.8,
+    "long_sinks/fwd_tc@096d815d8754": 508.7,
+    "decode_4k/decode@096d815d8754": 8120.7,
 }
+
+
+def workload_traffic(workload, kernel):
+    """The kernel's DRAM bytes per token-head from MEASURED_TRAFFIC at the
+    current kernel sources, with where the figure comes from."""
+    h = kernel_source_hash()
+    t = MEASURED_TRAFFIC.get(f"{workload}/{kernel}@{h}")
+    return {"traffic_B_per_token_head": t,
+            "traffic_source": f"ncu@{h}" if t is not None else f"none: no ncu capture of sources {h}"}
 
 
 def kernel_source_hash():
