@@ -46,7 +46,7 @@ struct FastArgs {
   __nv_bfloat16* o; float* lse;
   unsigned* err;
   long long wait_limit;                // bounded waits: SM clocks (0: the default)
-  int stall;                           // failure-path test: plant a stall in round 1
+  int stall;                           // failure-path test: the first staging round waits in vain
   float* save_p;                       // SAVE: [units][W+S+n_off][T] member probabilities
   float* save_dt;                      // SAVE: [units][n_off][T] row-score differences
   __half* save_q;                      // SAVE: [units][T][64] fp16 of RoPE(Q) * scale / 256

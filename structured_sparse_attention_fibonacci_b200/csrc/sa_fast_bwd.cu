@@ -53,7 +53,7 @@ struct FastBwdArgs {
   float* sink_k; float* sink_v;          // [units][n_tiles][S][64]
   unsigned* err;
   long long wait_limit;                // bounded waits: SM clocks (0: the default)
-  int stall;                           // failure-path test: plant a stall in round 1
+  int stall;                           // failure-path test: the first staging round waits in vain
   const float* ctx_p;                    // training context: [units][W+S+n_off][T] probabilities
   const float* ctx_dt;                   // ... and [units][n_off][T] row-score differences
   const float* beta;                     // log-prior on offset members [units][T], or nullptr

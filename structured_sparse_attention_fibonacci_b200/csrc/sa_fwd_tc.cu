@@ -48,7 +48,7 @@ struct TcFwdArgs {
   __nv_bfloat16* o; float* lse;
   unsigned* err;
   long long wait_limit;                // bounded waits: SM clocks (0: the default)
-  int stall;                           // failure-path test: plant a stall in round 1
+  int stall;                           // failure-path test: the first staging round waits in vain
   const float* beta;                   // log-prior on offset members [units][T], or nullptr
 };
 
