@@ -103,11 +103,13 @@ __device__ __forceinline__ void qk_mma(const uint32_t (&aq)[4][4], const uint32_
 // acc[0..7] (8 n tiles = 64 dims) += (A + Alo)(16 x 16 key rows) . V rows
 // kb .. kb + 15 (the weights as the bf16 pair split_bf16x2 makes); all eight B
 // fragments are loaded before the (independent) mma.
-__device__ __forceinline__ void pv_k16(uint32_t ring_u32, int RB, int kb, int lane,
+template <bool POW2>
+__device__ __forceinline__ void pv_k16(const Ring& ring, int kb, int lane,
                                        const uint32_t (&A)[4], const uint32_t (&Alo)[4],
                                        float (&acc)[8][4]) {
-  const int slot = (kb + (lane & 15)) & (RB - 1);
-  const uint32_t base = ring_u32 + (uint32_t)slot * 128u;
+  int slot = ring_slot<POW2>(ring, kb) + (lane & 15);
+  if (slot >= ring.rows) slot -= ring.rows;
+  const uint32_t base = ring.base + (uint32_t)slot * 128u;
   const int x = slot & 7, m = lane >> 4;
   uint32_t b[4][4];
 #pragma unroll
@@ -121,13 +123,15 @@ __device__ __forceinline__ void pv_k16(uint32_t ring_u32, int RB, int kb, int la
   }
 }
 
+// POW2: the ring's rows are a power of two (slots by a mask).
+template <bool POW2>
 __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ TcFwdArgs a) {
   constexpr int M = kFastM;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int RB = a.ring_rows, st = a.sc_stride;
-  const uint32_t ring_u32 = smem_u32(smem);
-  const uint32_t sink_u32 = ring_u32 + (uint32_t)RB * 128u;       // 16 rows, own swizzle atoms
+  const Ring ring = make_ring(smem_u32(smem), RB);
+  const Ring sinkr = make_ring(ring.base + (uint32_t)RB * 128u, 16);   // own swizzle atoms
   float* sc = reinterpret_cast<float*>(smem + (size_t)RB * 128 + 2048);
   float* inv_l = sc + (size_t)M * st;
   __shared__ OffGeo sg[SA_MAX_OFFSETS];
@@ -175,8 +179,8 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
   const int win_lo = floor16(i0 - W + 1);
 
   // ---------------- pass 1: scores ----------------
-  stage_tiles(stg, ring_u32, RB, &a.tmK, unit, win_lo, i0 + M);
-  if (S > 0) stage_tiles(stg, sink_u32, 16, &a.tmK, unit, 0, 16);
+  stage_tiles<POW2>(stg, ring, &a.tmK, unit, win_lo, i0 + M);
+  if (S > 0) stage_tiles<true>(stg, sinkr, &a.tmK, unit, 0, 16);
   if (stage_commit_wait(stg)) { stage_drain(stg); return; }
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt) {
@@ -185,8 +189,8 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
     const int n_nt = (qb + 16 - kr0) >> 3;
     for (int nt = 0; nt < n_nt; nt += 2) {      // n_nt is even
       uint32_t b0[2][4], b1[2][4];
-      qk_load(ring_u32, RB, kr0 + 8 * nt, lane, b0);
-      qk_load(ring_u32, RB, kr0 + 8 * nt + 8, lane, b1);
+      qk_load<POW2>(ring, kr0 + 8 * nt, lane, b0);
+      qk_load<POW2>(ring, kr0 + 8 * nt + 8, lane, b1);
       float c[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
       qk_mma(aq[mt], b0, c[0]);
       qk_mma(aq[mt], b1, c[1]);
@@ -202,7 +206,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
     for (int nt = 0; nt < ((S + 7) >> 3); ++nt) {
       float c[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t b[2][4];
-      qk_load(sink_u32, 16, 8 * nt, lane, b);
+      qk_load<true>(sinkr, 8 * nt, lane, b);
       qk_mma(aq[mt], b, c);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -226,7 +230,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
       const int lo_row = floor8(i0 - sg[last].lo - 1);
       if (lo_row < low) {
         __syncthreads();
-        stage_tiles(stg, ring_u32, RB, &a.tmK, unit, lo_row, min(hi, low));
+        stage_tiles<POW2>(stg, ring, &a.tmK, unit, lo_row, min(hi, low));
         if (stage_commit_wait(stg)) { stage_drain(stg); return; }
         low = lo_row;
       }
@@ -247,7 +251,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
             for (int e = 0; e < 4; ++e) cc[nt][e] = 0.f;
           if (two) {
 #pragma unroll
-            for (int nt = 0; nt < 3; ++nt) qk_load(ring_u32, RB, rb + 8 * nt, lane, b[nt]);
+            for (int nt = 0; nt < 3; ++nt) qk_load<POW2>(ring, rb + 8 * nt, lane, b[nt]);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
@@ -256,7 +260,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
                         b[nt][ks >> 1][2 * (ks & 1) + 1]);
           } else {                               // w == 0: row a only, two n tiles
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) qk_load(ring_u32, RB, rb + 8 * nt, lane, b[nt]);
+            for (int nt = 0; nt < 2; ++nt) qk_load<POW2>(ring, rb + 8 * nt, lane, b[nt]);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
 #pragma unroll
@@ -358,8 +362,8 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
   const bool bd_c2 = (g & 1) && tq == (g >> 1);
   const bool bd_c3 = (g & 1) && g < 7 && tq == ((g + 1) >> 1);
   const bool bd_a2 = g == 7 && tq == 0;
-  stage_tiles(stg, ring_u32, RB, &a.tmV, unit, win_lo, i0 + M);
-  if (S > 0) stage_tiles(stg, sink_u32, 16, &a.tmV, unit, 0, 16);
+  stage_tiles<POW2>(stg, ring, &a.tmV, unit, win_lo, i0 + M);
+  if (S > 0) stage_tiles<true>(stg, sinkr, &a.tmV, unit, 0, 16);
   if (stage_commit_wait(stg)) { stage_drain(stg); return; }
   float acc[2][8][4];
 #pragma unroll
@@ -388,7 +392,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
           const float v1 = (lag0 - 1 >= 0 && lag0 - 1 < W) ? er[lag0 - 1] : 0.f;
           split_bf16x2(v0, v1, A[h + 2 * p], Al[h + 2 * p]);
         }
-      pv_k16(ring_u32, RB, kb, lane, A, Al, acc[mt]);
+      pv_k16<POW2>(ring, kb, lane, A, Al, acc[mt]);
     }
     if (S > 0) {
       uint32_t A[4], Al[4];
@@ -401,7 +405,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
           split_bf16x2(s0 < S ? er[W + s0] : 0.f, s0 + 1 < S ? er[W + s0 + 1] : 0.f, A[h + 2 * p],
                        Al[h + 2 * p]);
         }
-      pv_k16(sink_u32, 16, 0, lane, A, Al, acc[mt]);
+      pv_k16<true>(sinkr, 0, lane, A, Al, acc[mt]);
     }
   }
   {
@@ -417,7 +421,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
       const int lo_row = floor8(i0 - sg[last].lo - 1);
       if (lo_row < low) {
         __syncthreads();
-        stage_tiles(stg, ring_u32, RB, &a.tmV, unit, lo_row, min(hi, low));
+        stage_tiles<POW2>(stg, ring, &a.tmV, unit, lo_row, min(hi, low));
         if (stage_commit_wait(stg)) { stage_drain(stg); return; }
         low = lo_row;
       }
@@ -441,7 +445,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
           split_bf16x2(bd_a2 ? sl : 0.f, 0.f, A[2], Al[2]);
           split_bf16x2(bd_lo_c1 ? dh : (bd_c3 ? sh : 0.f), bd_lo_c1 ? sh : (bd_c2 ? dh : 0.f), A[3],
                        Al[3]);
-          pv_k16(ring_u32, RB, kb, lane, A, Al, acc[mt]);
+          pv_k16<POW2>(ring, kb, lane, A, Al, acc[mt]);
           if (two) {
             // the 17th row (row a of query 15) as an 8-row k step
             uint32_t a1, a1l;
@@ -450,7 +454,7 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
               uint32_t b[4];
-              ldsm_x4_t(ring_u32 + swz_off(row, RB, 4 * hh + (lane >> 3)), b);
+              ldsm_x4_t(swz_addr<POW2>(ring, row, 4 * hh + (lane >> 3)), b);
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
                 mma_bf16_k8(acc[mt][4 * hh + i], 0u, a1, b[i]);
@@ -485,9 +489,35 @@ __global__ void __launch_bounds__(kFastM, 4) k_fwd_tc(const __grid_constant__ Tc
 
 __device__ unsigned g_fwd_tc_err;   // error bits as listed in sa_stage.cuh
 
+// CTAs of `smem` dynamic bytes that share one SM's 228 KB (1 KB reserved per
+// CTA plus about 1 KB of static shared memory), at most the 4 of the
+// launch bounds.
+int ctas_per_sm(size_t smem) {
+  const size_t per = smem + 2048;
+  return (int)std::min<size_t>(4, (size_t)(228 * 1024) / per);
+}
+
+size_t tc_smem_bytes(const Problem& pb, int rr, int st) {
+  return 1024 + (size_t)rr * 128 + 2048 + (size_t)kFastM * st * sizeof(float) +
+         kFastM * sizeof(float);
+}
+
+// Ring rows: at least the window round (M + W - 1 rows from a 16-aligned
+// start, so M + W + 15).  A power of two (slots by a mask) unless a multiple
+// of 16 fits more CTAs per SM; that ring then grows while the CTA count
+// holds (more far offsets per staging round).  Measured on B200 (B=1 H=16
+// T=32768, 4 sinks): W = 64 gains 16 % (3 CTAs per SM instead of 2) and
+// W = 128 38 % (2 instead of 1); where the count is the same the
+// power-of-two ring is 5-9 % faster than one indexed by a modulo.
 int tc_ring_rows(const Problem& pb) {
-  int rr = 32;
-  while (rr < std::max(kFastM + pb.W + 15, kFastM + 24)) rr *= 2;
+  const int st = (pb.W + pb.S + pb.n_off) | 1;
+  const int need = std::max(kFastM + pb.W + 15, kFastM + 24);
+  int p2 = 32;
+  while (p2 < need) p2 *= 2;
+  int rr = (need + 15) & ~15;
+  const int ctas = ctas_per_sm(tc_smem_bytes(pb, rr, st));
+  if (ctas_per_sm(tc_smem_bytes(pb, p2, st)) >= ctas) return p2;
+  while (rr + 16 <= 512 && ctas_per_sm(tc_smem_bytes(pb, rr + 16, st)) == ctas) rr += 16;
   return rr;
 }
 
@@ -498,8 +528,7 @@ size_t tc_fwd_smem(const Problem& pb, int* ring_rows, int* sc_stride) {
   const int st = (pb.W + pb.S + pb.n_off) | 1;
   if (ring_rows) *ring_rows = rr;
   if (sc_stride) *sc_stride = st;
-  return 1024 + (size_t)rr * 128 + 2048 + (size_t)kFastM * st * sizeof(float) +
-         kFastM * sizeof(float);
+  return tc_smem_bytes(pb, rr, st);
 }
 
 bool tc_fwd_supported(const Problem& pb) {
@@ -507,18 +536,11 @@ bool tc_fwd_supported(const Problem& pb) {
          tc_fwd_smem(pb, nullptr, nullptr) <= 200 * 1024;
 }
 
-// CTAs of `smem` dynamic bytes that share one SM's 228 KB (1 KB reserved per
-// CTA plus about 1 KB of static shared memory), at most the 4 of the
-// launch bounds.
-static int ctas_per_sm(size_t smem) {
-  const size_t per = smem + 2048;
-  return (int)std::min<size_t>(4, (size_t)(228 * 1024) / per);
-}
-
 // Measured on B200 (B=1 H=16 T=32768 d=64, 4 sinks, alpha = 1 and 1.1234,
-// windows 16..128): the CUDA-core forward is faster up to W = 40 (by 4-17%),
-// this one from W = 48 (by 2-4% at 48..56, 8-27% at 64..112); at W = 128 its
-// ring leaves it one CTA per SM and it is the slower (1.02 vs 0.83 ms).
+// windows 16..128): the CUDA-core forward is faster up to W = 40 (by 3-14 %),
+// this one from W = 48 (by 1-8 % at 48..56, 14-26 % at 64..128).  Where its
+// shared memory would leave it one CTA per SM while the CUDA-core forward
+// keeps two (W >= 160 with 15 offsets), it is not taken.
 bool tc_fwd_preferred(const Problem& pb) {
   if (!tc_fwd_supported(pb) || pb.W < 48) return false;
   const int tc = ctas_per_sm(tc_fwd_smem(pb, nullptr, nullptr));
@@ -549,12 +571,15 @@ cudaError_t launch_fwd_tc(const Problem& pb, const FwdPtrs& p, void* keys_ws, cu
   if ((e = launch_rope_rows(p.k, p.rope, pb.T, pb.units() * pb.T, kKeyStage, keys_ws, st,
                             "rope_keys")) != cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(k_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem)) != cudaSuccess)
+  const bool pow2 = (a.ring_rows & (a.ring_rows - 1)) == 0;
+  if ((e = cudaFuncSetAttribute(pow2 ? k_fwd_tc<true> : k_fwd_tc<false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+      cudaSuccess)
     return e;
   const unsigned grid = (unsigned)((long long)pb.units() * a.n_tiles);
   trace_mark("fwd_tc", st, true);
-  k_fwd_tc<<<grid, kFastM, smem, st>>>(a);
+  if (pow2) k_fwd_tc<true><<<grid, kFastM, smem, st>>>(a);
+  else k_fwd_tc<false><<<grid, kFastM, smem, st>>>(a);
   trace_mark("fwd_tc", st, false);
   e = cudaGetLastError();
   if (e == cudaSuccess) *launches += 2;

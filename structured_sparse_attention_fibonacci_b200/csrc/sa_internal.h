@@ -84,7 +84,9 @@ cudaError_t launch_fwd_fast(const Problem& pb, const FwdPtrs& a, void* keys_ws, 
 bool tc_fwd_supported(const Problem& pb);
 // Where the tensor-core forward is the faster one: windows of 48 and more,
 // except where its shared memory leaves it one CTA per SM while the CUDA-core
-// forward keeps two (measured on B200; at W = 12 it runs 25% slower).
+// forward keeps two (measured on B200; at W = 12 it runs 25% slower).  Its
+// ring of staged rows is a power of two, or a multiple of 16 where that fits
+// more CTAs per SM (W = 64 and 128 with 15 offsets and 4 sinks).
 bool tc_fwd_preferred(const Problem& pb);
 size_t tc_fwd_smem(const Problem& pb, int* ring_rows, int* sc_stride);
 cudaError_t launch_fwd_tc(const Problem& pb, const FwdPtrs& a, void* keys_ws, cudaStream_t st,

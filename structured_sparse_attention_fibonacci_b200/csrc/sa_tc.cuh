@@ -3,7 +3,7 @@
 // 128-byte-swizzled row ring, and 3-D tensor-map (TMA) staging of 8-row boxes.
 //
 // Swizzled ring.  Row r of a 16-bit [T][64] array lives in slot
-// s = r & (RB - 1) (RB a power of two, >= 8) at byte s * 128, and its 16-byte
+// s = r mod rows (rows a multiple of 16) at byte s * 128, and its 16-byte
 // chunk c at position c ^ (s & 7): the layout the tensor copy writes with
 // 128-byte swizzling into a 1024-byte-aligned ring.  Eight consecutive rows
 // then put any one chunk in eight different bank groups, so an ldmatrix of
@@ -96,10 +96,41 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uin
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
-// Byte offset, within the ring, of 16-byte chunk `ch` of row `row`.
-__device__ __forceinline__ uint32_t swz_off(int row, int RB, int ch) {
-  const int slot = row & (RB - 1);
-  return (uint32_t)(slot * 128 + ((ch ^ (slot & 7)) << 4));
+// A ring of `rows` 128-byte slots at shared address `base`.  Slots are
+// rows modulo `rows`: with POW2 (rows a power of two) a mask; otherwise a
+// multiply-high by inv = floor((2^32 - 1) / rows) (the quotient is exact or
+// one short, which one subtraction corrects) after adding bias = 64 rows, a
+// multiple of rows that makes every row the kernels stage (at least
+// -(W + 143)) non-negative.
+struct Ring {
+  uint32_t base;
+  int rows;
+  uint32_t inv;
+  int bias;
+};
+
+__host__ __device__ __forceinline__ Ring make_ring(uint32_t base, int rows) {
+  Ring r;
+  r.base = base;
+  r.rows = rows;
+  r.inv = 0xFFFFFFFFu / (uint32_t)rows;
+  r.bias = 64 * rows;
+  return r;
+}
+
+template <bool POW2>
+__device__ __forceinline__ int ring_slot(const Ring& r, int row) {
+  if (POW2) return row & (r.rows - 1);
+  const uint32_t x = (uint32_t)(row + r.bias);
+  const int s = (int)(x - __umulhi(x, r.inv) * (uint32_t)r.rows);
+  return s >= r.rows ? s - r.rows : s;
+}
+
+// Shared address of 16-byte chunk `ch` of row `row`.
+template <bool POW2>
+__device__ __forceinline__ uint32_t swz_addr(const Ring& r, int row, int ch) {
+  const int slot = ring_slot<POW2>(r, row);
+  return r.base + (uint32_t)(slot * 128 + ((ch ^ (slot & 7)) << 4));
 }
 
 // One 8-row box of a 3-D [units][T][64] 16-bit tensor map (row coordinate may
@@ -115,30 +146,34 @@ __device__ __forceinline__ void tma_rows8(uint32_t dst, const CUtensorMap* map, 
 }
 
 // Register (thread 0) and issue the copies of rows [a, b) (multiples of 8,
-// b - a <= RB) of `unit` into the ring at ring_u32.  Completes on the round's
-// barrier (stage::stage_commit_wait).
-__device__ __forceinline__ void stage_tiles(Stager& s, uint32_t ring_u32, int RB,
-                                            const CUtensorMap* map, int unit, int a, int b) {
+// b - a <= ring rows) of `unit` into the ring (a box of 8 rows never wraps:
+// rows is a multiple of 8).  Completes on the round's barrier
+// (stage::stage_commit_wait).
+template <bool POW2>
+__device__ __forceinline__ void stage_tiles(Stager& s, const Ring& ring, const CUtensorMap* map,
+                                            int unit, int a, int b) {
 #ifdef SA_DEBUG_BOUNDS
-  if (b - a > RB || (a & 7) || (b & 7)) {   // beyond the ring, or not whole boxes: stage none
+  if (b - a > ring.rows || (a & 7) || (b & 7)) {   // beyond the ring, or not whole boxes
     if (threadIdx.x == 0) atomicOr(s.err, stage::kErrBounds);
     return;
   }
 #endif
-  stage::dbg_staged(s, RB, a, b);
+  stage::dbg_staged(s, ring.rows, a, b);
   if (threadIdx.x != 0 || a >= b) return;
   stage::mbar_expect_tx(s.bar, (uint32_t)(b - a) * 128u);
   for (int r = a; r < b; r += 8)
-    tma_rows8(ring_u32 + (uint32_t)((r & (RB - 1)) * 128), map, r, unit, s.bar);
+    tma_rows8(ring.base + (uint32_t)ring_slot<POW2>(ring, r) * 128u, map, r, unit, s.bar);
 }
 
 // B fragments of one n tile of A . X^T for 8 swizzled ring rows row0 ..
 // row0 + 7 of a 16-bit [T][64] array: k steps 0..3 (dims 16 ks ..) as
 // b[kp][0..1] (k step 2 kp) and b[kp][2..3] (k step 2 kp + 1).
-__device__ __forceinline__ void qk_load(uint32_t ring_u32, int RB, int row0, int lane,
+template <bool POW2>
+__device__ __forceinline__ void qk_load(const Ring& ring, int row0, int lane,
                                         uint32_t (&b)[2][4]) {
-  const int slot = (row0 + (lane & 7)) & (RB - 1);
-  const uint32_t base = ring_u32 + (uint32_t)slot * 128u;
+  int slot = ring_slot<POW2>(ring, row0) + (lane & 7);
+  if (slot >= ring.rows) slot -= ring.rows;
+  const uint32_t base = ring.base + (uint32_t)slot * 128u;
   const int x = slot & 7, m = lane >> 3;
   ldsm_x4(base + (uint32_t)((m ^ x) << 4), b[0]);
   ldsm_x4(base + (uint32_t)(((4 + m) ^ x) << 4), b[1]);
