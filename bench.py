@@ -241,14 +241,14 @@ def decode_bytes_per_token_head(wl, elt):
 # capture per entry; keyed by workload, kernel and the hash of the kernel
 # sources the capture ran (kernel_source_hash): a changed source reports null.
 MEASURED_TRAFFIC = {
-    "learned_train/bwd_q_fast@34cbcc80c5b6": 778.7,
-    "pi_gate_train/bwd_q_fast@34cbcc80c5b6": 545.7,
-    "paper_fwd/fwd_fast@34cbcc80c5b6": 494.7,
-    "extrap_4x/fwd_fast@34cbcc80c5b6": 495.9,
-    "pow2_extrap/fwd_fast@34cbcc80c5b6": 495.9,
-    "pi_skip/fwd_fast@34cbcc80c5b6": 491.3,
-    "long_sinks/fwd_tc@34cbcc80c5b6": 508.3,
-    "decode_4k/decode@34cbcc80c5b6": 8121.8,
+    "learned_train/bwd_q_fast@a3631b8328cf": 780.3,
+    "pi_gate_train/bwd_q_fast@a3631b8328cf": 545.8,
+    "paper_fwd/fwd_fast@a3631b8328cf": 494.4,
+    "extrap_4x/fwd_fast@a3631b8328cf": 496.1,
+    "pow2_extrap/fwd_fast@a3631b8328cf": 496.3,
+    "pi_skip/fwd_fast@a3631b8328cf": 492.1,
+    "long_sinks/fwd_tc@a3631b8328cf": 505.3,
+    "decode_4k/decode@a3631b8328cf": 8121.5,
 }
 
 
