@@ -198,6 +198,10 @@ FAST = [
     ("fast_pow2_t4096", (2, 1, 1, 4096, 64), 12, 0, [1.0, 1.5], POW2_4096),
     ("fast_off32_t4096", (1, 1, 1, 4096, 64), 12, 2, [1.5], OFF32),
     ("fast_off32_w64", (1, 1, 1, 2000, 64), 64, 4, [1.0], OFF32),
+    # rings of staged rows that are not a power of two (the mma.sync forward
+    # sizes its ring for CTAs per SM: 224 rows here, 272 at W = 128)
+    ("fast_w64_s4_ring224", (1, 1, 2, 700, 64), 64, 4, [1.37], FIB15),
+    ("fast_w128_ring272", (1, 1, 1, 1100, 64), 128, 0, [0.77], FIB15),
 ]
 
 
